@@ -1,0 +1,165 @@
+"""Integer oracle of the continuous-batching step loop with recompute preemption.
+
+TEST INFRASTRUCTURE ONLY (see oracle/__init__.py).
+
+Sources:
+  "vLLM 原理：PagedAttention 和 Continuous Batching", "vLLM 的调度 / 调度流程":
+      each iteration 1) releases the pages of finished requests and drops them
+      from the running set, 2) admits waiting requests while free pages exist,
+      allocating their pages, 3) runs one forward step over the running set,
+      4) appends each request's new token to its KV cache.
+      "Preemption（抢占）": when memory runs short a lower-priority request is
+      suspended, its pages freed, and it resumes later by recomputation (or
+      swap; only recompute is modelled here).
+      "Continuous Batching": requests join as they arrive and leave as soon as
+      they finish.
+  "大模型推理性能优化：PagedAttention与Continuous Batching原理与实践" §2.3: a global
+      request queue checked at every decode iteration; finished requests leave
+      at once and free their pages; new requests join the next iteration.
+
+Readings where the pages are silent or loose (listed in the design notes):
+  * queue discipline is first come, first served: arrivals join the tail in
+    (arrival step, id) order and admission takes the head (the printed loop's
+    list pop would take the newest; the prose describes a request queue);
+  * "has free pages" means the free list holds ceil((prompt + generated) / 16)
+    blocks for the head request; admission stops at the first that does not fit;
+  * the phase order within a step is retire, arrive, admit, grow, (device
+    work), then generated += 1; a request admitted in a step decodes in it;
+  * the preemption victim ("lower priority") is the most recently admitted
+    running request; it goes back to the waiting head keeping its generated
+    count; if the victim is the request that is growing, it is preempted and
+    the grow phase ends (an error if nothing else is running: the pool cannot
+    hold that request);
+  * prompt K/V is (re)written only for requests admitted this step that are
+    still running at its end.
+"""
+from __future__ import annotations
+
+from collections import deque
+
+from .block_manager import BMError, OracleBlockManager, blocks_for
+
+
+class OracleScheduler:
+    def __init__(self, bm: OracleBlockManager, arrival_step, prompt_len, output_len,
+                 max_blocks_per_seq: int):
+        n = len(arrival_step)
+        if not (len(prompt_len) == n and len(output_len) == n):
+            raise BMError("INVALID_ARG", "request arrays differ in length")
+        for i in range(n):
+            if arrival_step[i] < 0 or prompt_len[i] < 1 or output_len[i] < 1:
+                raise BMError("INVALID_ARG", f"request {i}")
+            if blocks_for(prompt_len[i] + output_len[i]) > max_blocks_per_seq:
+                raise BMError("CAPACITY", f"request {i} exceeds the table width")
+        self.bm = bm
+        self.arrival = [int(x) for x in arrival_step]
+        self.prompt = [int(x) for x in prompt_len]
+        self.output = [int(x) for x in output_len]
+        self.max_blocks = max_blocks_per_seq
+        self.n = n
+        self.generated = [0] * n
+        self.arrival_order = sorted(range(n), key=lambda i: (self.arrival[i], i))
+        self.next_arrival = 0
+        self.waiting: deque[int] = deque()
+        self.running: list[int] = []
+        self.n_finished = 0
+        self.step_idx = 0
+
+    def step(self) -> dict:
+        s = self.step_idx
+        self.step_idx += 1
+        bm = self.bm
+
+        # 1. retire finished requests, freeing their pages at once
+        finished = [r for r in self.running if self.generated[r] >= self.output[r]]
+        for r in finished:
+            bm.free(r)
+        self.running = [r for r in self.running if self.generated[r] < self.output[r]]
+        self.n_finished += len(finished)
+
+        # 2. arrivals join the waiting tail
+        while (self.next_arrival < self.n
+               and self.arrival[self.arrival_order[self.next_arrival]] <= s):
+            self.waiting.append(self.arrival_order[self.next_arrival])
+            self.next_arrival += 1
+
+        # 3. admit from the head while its pages fit
+        admitted = []
+        admit_len = {}
+        while self.waiting:
+            r = self.waiting[0]
+            total = self.prompt[r] + self.generated[r]
+            if blocks_for(total) > bm.num_free():
+                if not self.running:
+                    raise BMError("NO_BLOCKS", f"request {r} can never fit")
+                break
+            self.waiting.popleft()
+            bm.allocate(r, total)
+            self.running.append(r)
+            admitted.append(r)
+            admit_len[r] = total
+
+        # 4. grow every running request by one slot, preempting from the tail
+        decode_slot = {}
+        cow = []
+        preempted = []
+        i = 0
+        stop = False
+        while i < len(self.running) and not stop:
+            r = self.running[i]
+            while True:
+                try:
+                    slot, cs, cd = bm.append_slot(r)
+                except BMError as e:
+                    if e.status != "NO_BLOCKS":
+                        raise
+                    victim = self.running.pop()
+                    bm.free(victim)
+                    self.waiting.appendleft(victim)
+                    preempted.append(victim)
+                    if victim == r:
+                        if not self.running:
+                            raise BMError("NO_BLOCKS", f"request {r} cannot grow alone")
+                        stop = True
+                        break
+                    continue
+                decode_slot[r] = slot
+                if cs >= 0:
+                    cow.append((cs, cd))
+                break
+            i += 1
+
+        # 5. the step's device work, described by index arrays
+        running = list(self.running)
+        still = set(running)
+        prompt_seqs = [r for r in admitted if r in still]
+        prompt_slots = []
+        for r in prompt_seqs:
+            prompt_slots.extend(bm.slots(r, 0, admit_len[r]))
+        tables = []
+        for r in running:
+            tab = bm.table(r)
+            tables.append(tab + [-1] * (self.max_blocks - len(tab)))
+
+        # 6. every running request generated one token
+        for r in running:
+            self.generated[r] += 1
+
+        done = (self.n_finished == self.n)
+        return {
+            "step": s,
+            "done": int(done),
+            "running": running,
+            "seq_lens": [bm.seq_len(r) for r in running],
+            "block_tables": tables,
+            "decode_slots": [decode_slot[r] for r in running],
+            "prompt_seqs": prompt_seqs,
+            "prompt_lens": [admit_len[r] for r in prompt_seqs],
+            "prompt_slots": prompt_slots,
+            "cow": cow,
+            "admitted": admitted,
+            "preempted": preempted,
+            "finished": finished,
+            "num_waiting": len(self.waiting),
+            "num_free_blocks": bm.num_free(),
+        }

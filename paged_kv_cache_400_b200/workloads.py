@@ -1,0 +1,332 @@
+"""Seeded synthetic workloads shared by the tests, the benchmark and the oracle checks.
+
+This module only produces inputs: random values, sequence lengths, pool
+placements, block-manager scripts and request traces. It holds none of the
+method's arithmetic (no page counts, slots, tables or attention); the product
+path and the oracle each derive those from what is generated here.
+
+Values. Every tensor element is drawn from one counter-based generator, so any
+element can be rebuilt on any device from its coordinates alone:
+    h_n  = mix(key + n * 0x9E3779B97F4A7C15)      (SplitMix64, Steele, Lea and
+           Flood, "Fast Splittable Pseudorandom Number Generators", OOPSLA 2014,
+           whose output function is Stafford's "Mix13" 64-bit finaliser)
+    x_c  = (sum of the 8 bytes of h_2c and the low 4 bytes of h_2c+1 + 6) / 256 - 6
+x_c is an Irwin-Hall(12) variate: mean 0, variance ~1, in [-6, 6), an exact
+multiple of 1/256, so it is the same fp32 number on CPU and GPU and rounds to
+the same bf16 number. It stands in for the N(0, 1) draws the workloads ask for.
+
+Workloads (sizes follow the decode configurations they are named after):
+  tiny      fp32, 4 sequences of length {5, 16, 17, 33} after the append,
+            2 query = 2 KV heads, head_dim 64, 64-block pool, scale 1/8.
+  mha       Llama-2-7B-shaped: 32 = 32 heads, head_dim 128, bf16, batch 64,
+            lengths uniform in [128, 2048], 16384-block pool.
+  gqa       Llama-3-8B-shaped: 32 query / 8 KV heads, head_dim 128, bf16,
+            batch 256, lengths lognormal (median 1000, sigma 0.8) rounded and
+            clipped to [16, 8192], 32768-block pool.
+  prefix    32 sequences sharing a 1536-token prefix plus private suffixes
+            uniform in [0, 512]; 8 prompts (length uniform in [16, 1024], not a
+            multiple of 16) x 4 samples forking at a partial block;
+            32/8 heads, head_dim 128, bf16, 4096-block pool.
+  trace     2000 requests, Poisson(50) arrivals per step, prompts uniform in
+            [16, 1024], outputs geometric with mean 200 capped at 2048,
+            40000-block pool, 32/8 heads, head_dim 128, bf16.
+Physical placement is random: the block manager's initial free list is a
+seeded permutation of the pool.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+# ---------------------------------------------------------------------------
+# counter-based value generator (SplitMix64 output stream, Irwin-Hall sum)
+# ---------------------------------------------------------------------------
+_U64 = 1 << 64
+
+
+def _s64(x: int) -> int:
+    """Unsigned 64-bit constant as the int64 with the same bits."""
+    x &= _U64 - 1
+    return x - _U64 if x >= (1 << 63) else x
+
+
+_GAMMA = _s64(0x9E3779B97F4A7C15)
+_M1 = _s64(0xBF58476D1CE4E5B9)
+_M2 = _s64(0x94D049BB133111EB)
+
+
+def _shr(z: torch.Tensor, k: int) -> torch.Tensor:
+    """Logical right shift of int64 bit patterns."""
+    return (z >> k) & ((1 << (64 - k)) - 1)
+
+
+def _mix(z: torch.Tensor) -> torch.Tensor:
+    z = (z ^ _shr(z, 30)) * _M1
+    z = (z ^ _shr(z, 27)) * _M2
+    return z ^ _shr(z, 31)
+
+
+def _mix_int(z: int) -> int:
+    z &= _U64 - 1
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & (_U64 - 1)
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & (_U64 - 1)
+    return z ^ (z >> 31)
+
+
+def stream_key(*coords: int) -> int:
+    """Key of a value stream named by small non-negative integers."""
+    k = 0x243F6A8885A308D3
+    for c in coords:
+        k = _mix_int(k ^ (int(c) & (_U64 - 1)))
+    return _s64(k)
+
+
+def values(key: int, counters: torch.Tensor) -> torch.Tensor:
+    """Irwin-Hall(12) values (fp32) at the given int64 counters of stream `key`."""
+    n = counters.to(torch.int64) * 2
+    h1 = _mix(n * _GAMMA + key)
+    h2 = _mix((n + 1) * _GAMMA + key)
+    s = torch.zeros_like(h1)
+    for i in range(8):
+        s += _shr(h1, 8 * i) & 0xFF
+    for i in range(4):
+        s += _shr(h2, 8 * i) & 0xFF
+    return (s.to(torch.float32) + 6.0) / 256.0 - 6.0
+
+
+def value_block(key: int, shape, offset: int = 0, device="cpu",
+                dtype=torch.float32) -> torch.Tensor:
+    """Values at counters offset .. offset+prod(shape)-1, row-major in `shape`."""
+    n = int(np.prod(shape))
+    c = torch.arange(offset, offset + n, dtype=torch.int64, device=device)
+    return values(key, c).to(dtype).reshape(shape)
+
+
+TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+# value-stream tags
+TAG_POOL, TAG_Q, TAG_K, TAG_V = 1, 2, 3, 4
+TAG_TRACE_KV, TAG_TRACE_Q = 5, 6
+
+
+# ---------------------------------------------------------------------------
+# single-step decode workloads
+# ---------------------------------------------------------------------------
+@dataclass
+class DecodeCase:
+    """One decode step over a pool prepared by a block-manager script.
+
+    ops: block-manager operations run in order before the step:
+         ("allocate", seq, num_tokens), ("fork", parent, child), ("free", seq),
+         ("append", seq) (a token whose K/V is already in the pool).
+    batch: the decode batch, in order; each sequence appends one token (its
+         K/V are k_new[i], v_new[i]) and then attends over its whole length.
+    table_width: columns of the packed block tables.
+    """
+    name: str
+    seed: int
+    num_blocks: int
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    dtype: str
+    scale: float
+    free_order: np.ndarray
+    ops: list
+    batch: list
+    table_width: int
+    max_seq_len: int
+    info: dict = field(default_factory=dict)
+
+    @property
+    def pool_shape(self):
+        return (self.num_blocks, 2, self.num_kv_heads, 16, self.head_dim)
+
+    def make_pool(self, device="cpu", chunk_blocks: int = 1024) -> torch.Tensor:
+        """Initial pool contents (every slot holds a value, used or not)."""
+        pool = torch.empty(self.pool_shape, dtype=TORCH_DTYPE[self.dtype], device=device)
+        per_block = int(np.prod(self.pool_shape[1:]))
+        key = stream_key(self.seed, TAG_POOL)
+        for b0 in range(0, self.num_blocks, chunk_blocks):
+            b1 = min(b0 + chunk_blocks, self.num_blocks)
+            pool[b0:b1] = value_block(key, (b1 - b0,) + self.pool_shape[1:],
+                                      offset=b0 * per_block, device=device,
+                                      dtype=pool.dtype)
+        return pool
+
+    def pool_blocks(self, block_ids, device="cpu") -> torch.Tensor:
+        """Initial contents of selected blocks only, [n][2][Hkv][16][D]."""
+        per_block = int(np.prod(self.pool_shape[1:]))
+        key = stream_key(self.seed, TAG_POOL)
+        ids = torch.as_tensor(np.asarray(block_ids, dtype=np.int64), device=device)
+        c = ids[:, None] * per_block + torch.arange(per_block, device=device)[None, :]
+        return values(key, c).to(TORCH_DTYPE[self.dtype]).reshape(
+            (len(block_ids),) + self.pool_shape[1:])
+
+    def make_q(self, device="cpu") -> torch.Tensor:
+        return value_block(stream_key(self.seed, TAG_Q),
+                           (len(self.batch), self.num_heads, self.head_dim),
+                           device=device, dtype=TORCH_DTYPE[self.dtype])
+
+    def make_kv_new(self, device="cpu"):
+        shape = (len(self.batch), self.num_kv_heads, self.head_dim)
+        k = value_block(stream_key(self.seed, TAG_K), shape, device=device,
+                        dtype=TORCH_DTYPE[self.dtype])
+        v = value_block(stream_key(self.seed, TAG_V), shape, device=device,
+                        dtype=TORCH_DTYPE[self.dtype])
+        return k, v
+
+
+def _decode_case_from_lens(name, seed, lens_after, num_blocks, num_heads, num_kv_heads,
+                           head_dim, dtype, scale, table_width, max_seq_len, rng):
+    """Sequences 0..B-1 hold len-1 tokens of cached context, then append one."""
+    free_order = rng.permutation(num_blocks).astype(np.int32)
+    ops = [("allocate", b, int(n) - 1) for b, n in enumerate(lens_after)]
+    return DecodeCase(name=name, seed=seed, num_blocks=num_blocks, num_heads=num_heads,
+                      num_kv_heads=num_kv_heads, head_dim=head_dim, dtype=dtype,
+                      scale=scale, free_order=free_order, ops=ops,
+                      batch=list(range(len(lens_after))), table_width=table_width,
+                      max_seq_len=max_seq_len,
+                      info={"seq_lens_after_append": [int(x) for x in lens_after]})
+
+
+def tiny_case(seed: int = 0) -> DecodeCase:
+    rng = np.random.default_rng(seed)
+    return _decode_case_from_lens("tiny_fp32", seed, [5, 16, 17, 33], 64, 2, 2, 64,
+                                  "f32", 1.0 / 8.0, 4, 64, rng)
+
+
+def mha_case(seed: int = 0, batch: int = 64) -> DecodeCase:
+    rng = np.random.default_rng(seed + 101)
+    lens = rng.integers(128, 2048, size=batch, endpoint=True)
+    return _decode_case_from_lens("mha_llama2_7b", seed, lens, 16384, 32, 32, 128,
+                                  "bf16", 128 ** -0.5, 128, 2048, rng)
+
+
+def gqa_lens(rng, batch: int):
+    x = rng.lognormal(mean=np.log(1000.0), sigma=0.8, size=batch)
+    return np.clip(np.round(x), 16, 8192).astype(np.int64)
+
+
+def gqa_case(seed: int = 0, batch: int = 256) -> DecodeCase:
+    rng = np.random.default_rng(seed + 202)
+    lens = gqa_lens(rng, batch)
+    return _decode_case_from_lens("gqa_llama3_8b", seed, lens, 32768, 32, 8, 128,
+                                  "bf16", 128 ** -0.5, 512, 8192, rng)
+
+
+def custom_case(name, seed, lens_after, num_blocks, num_heads, num_kv_heads, head_dim,
+                dtype, table_width, max_seq_len, scale=None) -> DecodeCase:
+    """A decode step with caller-chosen lengths (edge cases, small variants)."""
+    rng = np.random.default_rng(seed + 303)
+    if scale is None:
+        scale = head_dim ** -0.5
+    return _decode_case_from_lens(name, seed, list(lens_after), num_blocks, num_heads,
+                                  num_kv_heads, head_dim, dtype, scale, table_width,
+                                  max_seq_len, rng)
+
+
+def prefix_case(seed: int = 0) -> DecodeCase:
+    """Shared prefix + parallel sampling (copy-on-write at a partial block)."""
+    rng = np.random.default_rng(seed + 404)
+    num_blocks = 4096
+    free_order = rng.permutation(num_blocks).astype(np.int32)
+    ops = []
+    # (i) one 1536-token prefix held by seq 10000, forked to 32 sequences, each
+    #     of which then grows a private suffix; the holder is released.
+    holder = 10000
+    ops.append(("allocate", holder, 1536))
+    for i in range(32):
+        ops.append(("fork", holder, i))
+    ops.append(("free", holder))
+    suffix = rng.integers(0, 512, size=32, endpoint=True)
+    for i in range(32):
+        ops.extend([("append", i)] * int(suffix[i]))
+    # (ii) 8 prompts of length not a multiple of 16, each sampled 4 times
+    #      (the prompt sequence is sample 0, forked three times).
+    plens = []
+    while len(plens) < 8:
+        n = int(rng.integers(16, 1024, endpoint=True))
+        if n % 16 != 0:
+            plens.append(n)
+    batch = list(range(32))
+    for j, n in enumerate(plens):
+        p = 100 + j
+        ops.append(("allocate", p, n))
+        batch.append(p)
+        for s in range(1, 4):
+            c = 200 + 4 * j + s
+            ops.append(("fork", p, c))
+            batch.append(c)
+    return DecodeCase(name="shared_prefix", seed=seed, num_blocks=num_blocks,
+                      num_heads=32, num_kv_heads=8, head_dim=128, dtype="bf16",
+                      scale=128 ** -0.5, free_order=free_order, ops=ops, batch=batch,
+                      table_width=136, max_seq_len=2176,
+                      info={"prefix_len": 1536, "suffix_lens": [int(x) for x in suffix],
+                            "prompt_lens": plens, "samples": 4})
+
+
+# ---------------------------------------------------------------------------
+# continuous-batching trace
+# ---------------------------------------------------------------------------
+TRACE_MAX_POS = 4096    # positions per request in the K/V value space
+TRACE_MAX_REQ = 1 << 16
+TRACE_MAX_STEP = 1 << 20
+
+
+@dataclass
+class TraceCase:
+    seed: int
+    arrival_step: np.ndarray
+    prompt_len: np.ndarray
+    output_len: np.ndarray
+    num_blocks: int
+    num_layers: int
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    dtype: str
+    scale: float
+    table_width: int
+
+    def kv_values(self, layer: int, reqs, positions, device="cpu"):
+        """K and V of token `positions[i]` of request `reqs[i]` in `layer`:
+        two [n][num_kv_heads][head_dim] tensors. The same (layer, request,
+        position) always gives the same values, so recomputed K/V after a
+        preemption are identical to the originals."""
+        per_tok = 2 * self.num_kv_heads * self.head_dim
+        r = torch.as_tensor(np.asarray(reqs, dtype=np.int64), device=device)
+        p = torch.as_tensor(np.asarray(positions, dtype=np.int64), device=device)
+        base = (r * TRACE_MAX_POS + p) * per_tok
+        c = base[:, None] + torch.arange(per_tok, device=device)[None, :]
+        x = values(stream_key(self.seed, TAG_TRACE_KV, layer), c).to(TORCH_DTYPE[self.dtype])
+        x = x.reshape(len(r), 2, self.num_kv_heads, self.head_dim)
+        return x[:, 0].contiguous(), x[:, 1].contiguous()
+
+    def q_values(self, layer: int, step: int, reqs, device="cpu"):
+        """Query of each request in `reqs` at (layer, step): [n][H][D]."""
+        per = self.num_heads * self.head_dim
+        r = torch.as_tensor(np.asarray(reqs, dtype=np.int64), device=device)
+        c = ((step * TRACE_MAX_REQ + r) * per)[:, None] + torch.arange(per, device=device)[None, :]
+        x = values(stream_key(self.seed, TAG_TRACE_Q, layer), c).to(TORCH_DTYPE[self.dtype])
+        return x.reshape(len(r), self.num_heads, self.head_dim)
+
+
+def trace_case(seed: int = 0, n_requests: int = 2000, rate: float = 50.0,
+               num_blocks: int = 40000, num_layers: int = 32) -> TraceCase:
+    rng = np.random.default_rng(seed + 505)
+    arrivals = []
+    step = 0
+    while len(arrivals) < n_requests:
+        k = int(rng.poisson(rate))
+        arrivals.extend([step] * k)
+        step += 1
+    arrivals = np.asarray(arrivals[:n_requests], dtype=np.int32)
+    prompt = rng.integers(16, 1024, size=n_requests, endpoint=True).astype(np.int32)
+    output = np.minimum(rng.geometric(1.0 / 200.0, size=n_requests), 2048).astype(np.int32)
+    return TraceCase(seed=seed, arrival_step=arrivals, prompt_len=prompt, output_len=output,
+                     num_blocks=num_blocks, num_layers=num_layers, num_heads=32,
+                     num_kv_heads=8, head_dim=128, dtype="bf16", scale=128 ** -0.5,
+                     table_width=192)
