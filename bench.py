@@ -1,0 +1,415 @@
+"""Benchmark: paged decode attention + cache append on the Llama-3-8B-shaped GQA
+decode step (32 query / 8 KV heads, head_dim 128, bf16, block 16, batch 256,
+lognormal lengths median 1000 sigma 0.8 clipped to [16, 8192], random block
+placement in a 32768-block pool).
+
+One step = one pass of the hot path over the batch: append the batch's new
+K/V into their slots (pa_reshape_and_cache), then split-KV paged decode with
+its partition reduce (pa_decode). Inputs are resident in HBM before timing;
+the KV read per step (~1.5 GB) is far larger than L2, so no flush is needed.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs its own independent batch (seed = rank): the
+path has no exchange step, so ranks share nothing but the barrier and the
+max-over-ranks timing ("weak" scaling). --impl reference times the fp64 CPU
+oracle on a bounded sample of the same workload (rank 0 only).
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode-attn tokens/s; KV-read HBM GB/s as fraction of ~8 TB/s peak"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "pa_decode_gqa_b256.md")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="bounded oracle sample for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_description(case):
+    lens = np.asarray(case.info["seq_lens_after_append"])
+    return {
+        "workload": "gqa_llama3_8b_decode: 32 q / 8 kv heads, head_dim 128, bf16, block_size 16, "
+                    "batch 256, seq_lens lognormal(median 1000, sigma 0.8) clipped [16, 8192], "
+                    "32768-block pool, random placement; step = cache append + split-KV decode",
+        "global_batch": None,
+        "seq_len_mean": float(lens.mean()),
+        "seq_len_max": int(lens.max()),
+        "tokens_in_cache": int(lens.sum()),
+        "l2": "no flush: inputs larger than L2 (KV read per step %.2f GB vs 126 MB L2)"
+              % (lens.sum() * 2 * case.num_kv_heads * case.head_dim * 2 / 1e9),
+    }
+
+
+def algorithmic_bytes(case, prep, partitions_per_seq, max_partitions):
+    """Bytes the step must move at minimum (the kernel's roofline traffic)."""
+    elt = 2
+    lens = prep.seq_lens.astype(np.int64)
+    B, H, Hkv, D = len(lens), case.num_heads, case.num_kv_heads, case.head_dim
+    kv = int(lens.sum()) * 2 * Hkv * D * elt                       # K and V rows read
+    qo = 2 * B * H * D * elt                                       # q read, out written
+    tables = int(((lens + 15) // 16).sum()) * 4 + B * 4            # table entries + lengths
+    split = int(sum(p for p in partitions_per_seq if p > 1)) * H * (D + 2) * 4 * 2  # partials w+r
+    append = 2 * 2 * B * Hkv * D * elt + B * 8                     # k/v read + written, slots
+    return {"kv": kv, "decode": kv + qo + tables + split, "append": append,
+            "step": kv + qo + tables + split + append}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML every 10 ms."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - reported in the JSON
+            self.err = repr(e)
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        p = self.nvml
+        while not self._stop.is_set():
+            try:
+                mhz = p.nvmlDeviceGetClockInfo(self.h, p.NVML_CLOCK_SM)
+                rs = p.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = "sampled during the timed region"
+        if not inside:
+            inside = self.samples[-5:]
+            note = "timed region shorter than the sampling period: last samples before its end"
+        reasons = set()
+        for _, _, rs in inside:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(m for _, m, _ in inside) if inside else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(inside), "note": note}
+
+
+def kernel_source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_400_b200", "csrc", "device")
+    for n in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(n.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """ncu DRAM bytes per launch recorded in profiles/, if taken on this source."""
+    try:
+        text = open(TRAFFIC_FILE).read()
+    except OSError:
+        return None, "no ncu summary"
+    m = re.search(r"kernel_source_digest:\s*([0-9a-f]+)", text)
+    t = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not (m and t):
+        return None, "summary lacks digest or traffic"
+    if m.group(1) != kernel_source_digest():
+        return None, "kernel changed since the ncu capture"
+    return int(t.group(1)), "ncu capture"
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(case, seconds, rng_seed=0):
+    """Times the oracle (as it stands) on whole sequences of the batch, one at a
+    time in random order, for about `seconds` of oracle work: its copy-on-write
+    copies, cache append and fp64 attention. Input generation (the generator's
+    pool blocks, q, k, v) and the oracle block-manager replay are outside the
+    timed part. Returns (sequences done, oracle seconds)."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from oracle_side import oracle_compute, oracle_indices, oracle_inputs
+    ost = oracle_indices(case)
+    order = np.random.default_rng(rng_seed).permutation(len(case.batch))
+    done, busy = 0, 0.0
+    while done < len(order) and busy < seconds:
+        x = oracle_inputs(case, ost, [int(order[done])])
+        t0 = time.perf_counter()
+        oracle_compute(x)
+        busy += time.perf_counter() - t0
+        done += 1
+    return done, busy
+
+
+def run_reference(args, rank, world):
+    from paged_kv_cache_400_b200 import workloads as wl
+    if rank != 0:
+        return
+    case = wl.gqa_case(args.seed)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from oracle_side import oracle_compute, oracle_indices, oracle_inputs
+    ost = oracle_indices(case)
+    rng = np.random.default_rng(1)
+    per_step = 2  # sequences per step: a bounded sample of the batch
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = [int(x) for x in rng.choice(len(case.batch), size=per_step, replace=False)]
+        x = oracle_inputs(case, ost, rows)
+        t0 = time.perf_counter()
+        oracle_compute(x)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = per_step * len(times) / total
+    cfg = workload_description(case)
+    cfg["global_batch"] = per_step
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{per_step} random sequences of the batch per step (their KV "
+                                   "gathered through the oracle block manager's tables), fp64"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, dist):
+    import torch
+
+    import paged_kv_cache_400_b200 as pk
+    from paged_kv_cache_400_b200 import workloads as wl
+    from paged_kv_cache_400_b200.scenario import prepare_decode_step
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    case = wl.gqa_case(args.seed + rank)
+    prep = prepare_decode_step(case)
+    B, H, D = len(case.batch), case.num_heads, case.head_dim
+    pool = case.make_pool(dev)
+    q = case.make_q(dev)
+    k, v = case.make_kv_new(dev)
+    slots = torch.from_numpy(prep.slot_mapping).to(dev)
+    bt = torch.from_numpy(prep.block_tables).to(dev)
+    sl = torch.from_numpy(prep.seq_lens).to(dev)
+    out = torch.empty_like(q)
+    ws = pk.alloc_workspace(B, H, pool, case.max_seq_len)
+    S = pk.pa_decode_partition_tokens(B, H, pool, case.max_seq_len)
+    parts = [(int(n) + S - 1) // S for n in prep.seq_lens]
+    nbytes = algorithmic_bytes(case, prep, parts, max(parts))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        pk.pa_reshape_and_cache(k, v, pool, slots)
+        pk.pa_decode(out, q, pool, bt, sl, case.scale, case.max_seq_len, ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    assert pk.pa_get_device_error() == 0
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    t_start.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        pk.pa_reshape_and_cache(k, v, pool, slots)
+        ev[i][1].record(stream)
+        pk.pa_decode(out, q, pool, bt, sl, case.scale, case.max_seq_len, ws)
+        ev[i][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.perf_counter()
+    if dist is not None:
+        dist.barrier()
+    sampler.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    append_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    decode_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    assert pk.pa_get_device_error() == 0
+
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    value = world * B / (ms_per_step / 1e3)
+
+    # ---- e2e: host buffers through the public API, copies inside the region
+    E = args.e2e_steps or min(K, 100)
+    pin = lambda t: t.cpu().pin_memory()
+    h_q, h_k, h_v = pin(q), pin(k), pin(v)
+    h_slots = pin(slots)
+    h_bt, h_sl = pin(bt), pin(sl)
+    h_out = torch.empty_like(out, device="cpu").pin_memory()
+    bt_np, sl_np = h_bt.numpy(), h_sl.numpy()
+    batch = np.asarray(case.batch, np.int64)
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_bt, h_sl))
+    d2h = h_out.numel() * h_out.element_size()
+    for i in range(3 + E):
+        if i == 3:
+            if dist is not None:
+                dist.barrier()
+            torch.cuda.synchronize()
+            e0 = time.perf_counter()
+        prep.bm.pack(batch, case.table_width, bt_np, sl_np, None)   # host tables (C ABI)
+        q.copy_(h_q, non_blocking=True)
+        k.copy_(h_k, non_blocking=True)
+        v.copy_(h_v, non_blocking=True)
+        slots.copy_(h_slots, non_blocking=True)
+        bt.copy_(h_bt, non_blocking=True)
+        sl.copy_(h_sl, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+        stream.synchronize()
+    e1 = time.perf_counter()
+    e2e_s = (e1 - e0) / E
+    if dist is not None:
+        t = torch.tensor([e2e_s], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+
+    if rank != 0:
+        return
+    peak, peak_src = measured_peak()
+    dec_avg_ms = sum(decode_ms) / K
+    achieved = nbytes["decode"] / (dec_avg_ms / 1e3) / 1e9
+    traffic, traffic_src = recorded_traffic()
+    kv_gbs = nbytes["kv"] / (ms_per_step / 1e3) / 1e9
+    cfg = workload_description(case)
+    cfg["global_batch"] = B * world
+    cfg["parallelism"] = f"dp{world} independent replicas (no exchange step)"
+    cfg["partition_tokens"] = S
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": cfg,
+        "kv_read_gbs": kv_gbs, "kv_frac_of_8tbs": kv_gbs / NOMINAL_HBM_GBS,
+        "kv_frac_of_measured": kv_gbs / peak,
+        "roofline": {"kernel": "pa_decode (split-KV partition kernel + partition reduce)",
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_src,
+                     "traffic": traffic, "traffic_source": traffic_src,
+                     "algorithmic_bytes_per_launch": nbytes["decode"],
+                     "avg_launch_ms": dec_avg_ms, "append_avg_ms": sum(append_ms) / K},
+        "gpu_launches": K * (2 + (1 if max(parts) > 1 else 0)),
+        "clocks": sampler.summary(wall0, wall1),
+        "e2e": {"value": world * B / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "note": "per step: host table packing (pa_bm_pack), H2D of q/k/v/slots/tables/lens "
+                        "from pinned memory, append + decode, D2H of out, stream sync"},
+        "library": os.path.relpath(pk.library_path(), ROOT),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        done, el = oracle_sample(case, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": done / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{done} of {B} sequences (random order), one decode token each: oracle "
+                      f"gather through its own block tables + fp64 attention, {el:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if args.impl == "reference" and rank != 0:
+        return  # the CPU oracle runs on rank 0 only
+    if world > 1 and args.impl == "ours":
+        import datetime
+
+        import torch
+        import torch.distributed as dist_mod
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = dist_mod
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

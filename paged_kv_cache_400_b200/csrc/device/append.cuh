@@ -1,0 +1,60 @@
+// Cache append ("scatter" of each new token's K/V into its slot) and whole-block
+// copy for copy-on-write.
+//
+// "大模型推理性能优化：PagedAttention与Continuous Batching原理与实践" §2.2 names the
+// scatter of new K/V into scattered pages as one of the two memory operations
+// PagedAttention kernels must do well; "vLLM 原理" / 工作原理 §2 gives the
+// position -> (page, row) mapping. Both kernels are plain 16-byte copies: every
+// thread moves one 16-byte chunk, consecutive threads take consecutive chunks
+// of one (token, K|V, head) row, so each row is one coalesced run on both sides.
+#pragma once
+
+#include "common.cuh"
+
+namespace pagedkv {
+
+// One thread per 16-byte chunk; item i = ((t * 2 + kv) * Hkv + h) * C + c,
+// C = chunks per (token, head) row.
+__global__ void __launch_bounds__(256)
+append_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, uint4* __restrict__ pool,
+              const int64_t* __restrict__ slots, int32_t num_tokens, int32_t num_kv_heads,
+              int32_t chunks_per_row, int64_t num_slots) {
+  const int64_t total = (int64_t)num_tokens * 2 * num_kv_heads * chunks_per_row;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const int32_t c = (int32_t)(i % chunks_per_row);
+    int64_t r = i / chunks_per_row;
+    const int32_t h = (int32_t)(r % num_kv_heads);
+    r /= num_kv_heads;
+    const int32_t kv = (int32_t)(r & 1);
+    const int64_t t = r >> 1;
+    const int64_t s = __ldg(slots + t);
+    if (s < 0) continue;  // padding
+    if (s >= num_slots) {
+      if (c == 0 && h == 0 && kv == 0) raise_device_error(PA_DEVERR_SLOT);
+      continue;
+    }
+    const int64_t blk = s >> 4;
+    const int32_t row = (int32_t)(s & 15);
+    const uint4* src = (kv ? v : k) + (t * num_kv_heads + h) * chunks_per_row + c;
+    uint4* dst = pool + (((blk * 2 + kv) * num_kv_heads + h) * 16 + row) * chunks_per_row + c;
+    *dst = __ldg(src);
+  }
+}
+
+// One CTA per pair; the CTA copies the whole block as 16-byte chunks.
+__global__ void __launch_bounds__(256)
+copy_blocks_kernel(uint4* __restrict__ pool, const int32_t* __restrict__ src,
+                   const int32_t* __restrict__ dst, int32_t num_blocks, int64_t chunks_per_block) {
+  const int32_t s = src[blockIdx.x];
+  const int32_t d = dst[blockIdx.x];
+  if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) {
+    if (threadIdx.x == 0) raise_device_error(PA_DEVERR_BLOCK);
+    return;
+  }
+  const uint4* from = pool + (int64_t)s * chunks_per_block;
+  uint4* to = pool + (int64_t)d * chunks_per_block;
+  for (int64_t i = threadIdx.x; i < chunks_per_block; i += blockDim.x) to[i] = from[i];
+}
+
+}  // namespace pagedkv

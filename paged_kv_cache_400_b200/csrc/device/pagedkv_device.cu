@@ -1,0 +1,235 @@
+// C-ABI device entry points of libpagedkv.so: argument checks, kernel choice,
+// launches. All kernels live in this one translation unit so they share the
+// per-device error word without relocatable device code.
+#include <cmath>
+#include <cstring>
+
+#include "../host/errors.hpp"
+#include "append.cuh"
+#include "common.cuh"
+#include "decode_common.cuh"
+#include "decode_generic.cuh"
+#include "decode_staged.cuh"
+
+using pagedkv::fail;
+
+namespace {
+
+constexpr int32_t kNumSMs = 148;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_size(int32_t dtype) { return dtype == PA_BF16 ? 2 : 4; }
+
+pa_status check_pool(const pa_pool_desc& pool, const char* fn) {
+  if (pool.block_size != PA_BLOCK_SIZE)
+    return fail(PA_ERR_UNSUPPORTED, "%s: block_size %d (only 16)", fn, pool.block_size);
+  if (pool.dtype != PA_F32 && pool.dtype != PA_BF16)
+    return fail(PA_ERR_UNSUPPORTED, "%s: dtype %d", fn, pool.dtype);
+  if (pool.head_dim != 64 && pool.head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "%s: head_dim %d (64 or 128)", fn, pool.head_dim);
+  if (pool.num_blocks <= 0 || pool.num_kv_heads <= 0)
+    return fail(PA_ERR_INVALID_ARG, "%s: num_blocks %d, num_kv_heads %d", fn, pool.num_blocks,
+                pool.num_kv_heads);
+  return PA_OK;
+}
+
+pa_status launch_status(const char* fn) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "%s: launch failed: %s", fn, cudaGetErrorString(e));
+  return PA_OK;
+}
+
+int32_t partition_tokens_for(int32_t num_seqs, const pa_pool_desc& pool, int32_t max_seq_len) {
+  // 512-token partitions; halve while the grid would not give every SM a few
+  // CTAs, down to 128.
+  int32_t S = 512;
+  const int64_t pairs = (int64_t)num_seqs * pool.num_kv_heads;
+  while (S > 128 && pairs * ((max_seq_len + S - 1) / S) < 4 * kNumSMs) S /= 2;
+  return S;
+}
+
+struct WorkspaceLayout {
+  size_t acc_bytes, ml_offset, total;
+  int32_t partitions;
+};
+
+WorkspaceLayout workspace_layout(int32_t num_seqs, int32_t num_heads, const pa_pool_desc& pool,
+                                 int32_t max_seq_len) {
+  WorkspaceLayout w{0, 0, 0, 0};
+  const int32_t S = partition_tokens_for(num_seqs, pool, max_seq_len);
+  w.partitions = (max_seq_len + S - 1) / S;
+  if (w.partitions <= 1) return w;
+  const size_t units = (size_t)num_seqs * num_heads * w.partitions;
+  w.acc_bytes = units * pool.head_dim * sizeof(float);
+  w.ml_offset = (w.acc_bytes + 255) & ~(size_t)255;
+  w.total = w.ml_offset + units * 2 * sizeof(float);
+  return w;
+}
+
+template <typename T, int D>
+pa_status launch_generic(const pagedkv::DecodeParams& p, cudaStream_t st) {
+  dim3 grid(p.max_partitions, p.num_kv_heads, p.num_seqs);
+  const int G = p.group;
+  if (G <= 1) pagedkv::decode_generic_kernel<T, D, 1><<<grid, 128, 0, st>>>(p);
+  else if (G <= 2) pagedkv::decode_generic_kernel<T, D, 2><<<grid, 128, 0, st>>>(p);
+  else if (G <= 4) pagedkv::decode_generic_kernel<T, D, 4><<<grid, 128, 0, st>>>(p);
+  else if (G <= 8) pagedkv::decode_generic_kernel<T, D, 8><<<grid, 128, 0, st>>>(p);
+  else pagedkv::decode_generic_kernel<T, D, 16><<<grid, 128, 0, st>>>(p);
+  pa_status s = launch_status("pa_decode");
+  if (s != PA_OK || p.max_partitions <= 1) return s;
+  pagedkv::partition_reduce_kernel<T, D><<<dim3(p.num_heads, p.num_seqs), D, 0, st>>>(p);
+  return launch_status("pa_decode (reduce)");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_NO_BLOCKS: return "no free blocks";
+    case PA_ERR_UNKNOWN_SEQ: return "unknown sequence";
+    case PA_ERR_DEVICE_BOUNDS: return "device index out of bounds";
+    case PA_ERR_SEQ_EXISTS: return "sequence exists";
+    case PA_ERR_CAPACITY: return "capacity exceeded";
+    case PA_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+const char* pa_last_error(void) { return pagedkv::last_error_slot().c_str(); }
+
+pa_status pa_reshape_and_cache(const void* k, const void* v, void* kv_pool,
+                               const int64_t* slot_mapping, int32_t num_tokens,
+                               pa_pool_desc pool, void* stream) {
+  pa_status s = check_pool(pool, "pa_reshape_and_cache");
+  if (s != PA_OK) return s;
+  if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "pa_reshape_and_cache: num_tokens %d", num_tokens);
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !kv_pool || !slot_mapping)
+    return fail(PA_ERR_INVALID_ARG, "pa_reshape_and_cache: NULL pointer");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(kv_pool))
+    return fail(PA_ERR_INVALID_ARG, "pa_reshape_and_cache: k, v and kv_pool must be 16-byte aligned");
+  const int32_t chunks = (int32_t)(pool.head_dim * elem_size(pool.dtype) / 16);
+  const int64_t total = (int64_t)num_tokens * 2 * pool.num_kv_heads * chunks;
+  const int64_t want = (total + 255) / 256;
+  const int32_t grid = (int32_t)(want < 65535 * 16 ? want : 65535 * 16);
+  pagedkv::append_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v),
+      reinterpret_cast<uint4*>(kv_pool), slot_mapping, num_tokens, pool.num_kv_heads, chunks,
+      (int64_t)pool.num_blocks * PA_BLOCK_SIZE);
+  return launch_status("pa_reshape_and_cache");
+}
+
+int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_heads, pa_pool_desc pool,
+                                   int32_t max_seq_len) {
+  (void)num_heads;
+  if (num_seqs < 0 || max_seq_len < 0 || pool.num_kv_heads <= 0) return 0;
+  return partition_tokens_for(num_seqs, pool, max_seq_len);
+}
+
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, pa_pool_desc pool,
+                                int32_t max_seq_len) {
+  if (num_seqs <= 0 || num_heads <= 0 || max_seq_len <= 0 || pool.num_kv_heads <= 0 ||
+      pool.head_dim <= 0)
+    return 0;
+  return workspace_layout(num_seqs, num_heads, pool, max_seq_len).total;
+}
+
+pa_status pa_decode(void* out, const void* q, const void* kv_pool, const int32_t* block_tables,
+                    int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t num_seqs,
+                    int32_t num_heads, float scale, pa_pool_desc pool, void* workspace,
+                    size_t workspace_bytes, int32_t max_seq_len, void* stream) {
+  pa_status s = check_pool(pool, "pa_decode");
+  if (s != PA_OK) return s;
+  if (num_seqs < 0 || num_heads <= 0 || max_blocks_per_seq <= 0 || max_seq_len < 0)
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: num_seqs %d, num_heads %d, max_blocks %d, max_seq_len %d",
+                num_seqs, num_heads, max_blocks_per_seq, max_seq_len);
+  if (num_heads % pool.num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: num_heads %d not a multiple of num_kv_heads %d", num_heads,
+                pool.num_kv_heads);
+  const int32_t G = num_heads / pool.num_kv_heads;
+  if (G > 16) return fail(PA_ERR_UNSUPPORTED, "pa_decode: head group %d > 16", G);
+  if (num_seqs > 65535) return fail(PA_ERR_UNSUPPORTED, "pa_decode: num_seqs %d > 65535", num_seqs);
+  if ((int64_t)max_seq_len > (int64_t)max_blocks_per_seq * PA_BLOCK_SIZE)
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: max_seq_len %d > max_blocks_per_seq * 16", max_seq_len);
+  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "pa_decode: scale is not finite");
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !kv_pool || !block_tables || !seq_lens)
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: NULL pointer");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(kv_pool))
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: out, q and kv_pool must be 16-byte aligned");
+  const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, pool, max_seq_len > 0 ? max_seq_len : 1);
+  if (w.total > 0 && (!workspace || workspace_bytes < w.total))
+    return fail(PA_ERR_WORKSPACE, "pa_decode: workspace %zu bytes at %p, need %zu", workspace_bytes,
+                workspace, w.total);
+  if (w.total > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: workspace must be 256-byte aligned");
+
+  pagedkv::DecodeParams p;
+  p.out = out;
+  p.q = q;
+  p.pool = kv_pool;
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.ws_acc = reinterpret_cast<float*>(workspace);
+  p.ws_ml = w.total ? reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + w.ml_offset) : nullptr;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_seqs = num_seqs;
+  p.num_heads = num_heads;
+  p.num_kv_heads = pool.num_kv_heads;
+  p.group = G;
+  p.num_blocks = pool.num_blocks;
+  p.max_seq_len = max_seq_len;
+  p.partition_tokens = partition_tokens_for(num_seqs, pool, max_seq_len > 0 ? max_seq_len : 1);
+  p.max_partitions = w.partitions > 0 ? w.partitions : 1;
+  p.scale_log2 = scale * pagedkv::kLog2e;
+  cudaStream_t st = (cudaStream_t)stream;
+
+  if (pool.dtype == PA_BF16 && pool.head_dim == 128) {
+    pa_status r = pagedkv::launch_staged_bf16_d128(p, st);
+    if (r != PA_ERR_UNSUPPORTED) return r;
+  }
+  if (pool.dtype == PA_BF16) {
+    return pool.head_dim == 128 ? launch_generic<__nv_bfloat16, 128>(p, st)
+                                : launch_generic<__nv_bfloat16, 64>(p, st);
+  }
+  return pool.head_dim == 128 ? launch_generic<float, 128>(p, st) : launch_generic<float, 64>(p, st);
+}
+
+pa_status pa_copy_blocks(void* kv_pool, const int32_t* src, const int32_t* dst, int32_t n,
+                         pa_pool_desc pool, void* stream) {
+  pa_status s = check_pool(pool, "pa_copy_blocks");
+  if (s != PA_OK) return s;
+  if (n < 0) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: n %d", n);
+  if (n == 0) return PA_OK;
+  if (!kv_pool || !src || !dst) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: NULL pointer");
+  if (!aligned16(kv_pool)) return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks: kv_pool must be 16-byte aligned");
+  const int64_t chunks = (int64_t)2 * pool.num_kv_heads * PA_BLOCK_SIZE * pool.head_dim *
+                         (int64_t)elem_size(pool.dtype) / 16;
+  pagedkv::copy_blocks_kernel<<<n, 256, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<uint4*>(kv_pool), src, dst, pool.num_blocks, chunks);
+  return launch_status("pa_copy_blocks");
+}
+
+pa_status pa_get_device_error(uint32_t* flags, void* stream) {
+  if (!flags) return fail(PA_ERR_INVALID_ARG, "pa_get_device_error: flags is NULL");
+  void* addr = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&addr, pagedkv::g_error_word);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_get_device_error: %s", cudaGetErrorString(e));
+  cudaStream_t st = (cudaStream_t)stream;
+  uint32_t v = 0;
+  e = cudaMemcpyAsync(&v, addr, sizeof(v), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(addr, 0, sizeof(uint32_t), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_get_device_error: %s", cudaGetErrorString(e));
+  *flags = v;
+  return v ? PA_ERR_DEVICE_BOUNDS : PA_OK;
+}
+
+}  // extern "C"

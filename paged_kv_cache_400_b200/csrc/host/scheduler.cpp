@@ -1,0 +1,240 @@
+// Continuous-batching step loop with recompute-mode preemption.
+//
+// Follows "vLLM 原理：PagedAttention 和 Continuous Batching" / "vLLM 的调度 / 调度流程"
+// (each iteration: release finished requests' pages, admit waiting requests
+// while pages are free, run one step, append each request's token) and
+// "Preemption（抢占）" (when memory runs short a lower-priority request is
+// suspended, its pages freed, and it later resumes by recomputation), and
+// "大模型推理性能优化：PagedAttention与Continuous Batching原理与实践" §2.3 (a global
+// request queue; finished requests leave at once; new ones join the next
+// iteration). The step rules the pages leave open are fixed in pagedkv.h
+// (pa_sched_create): FCFS queue, admission while ceil((prompt+generated)/16)
+// blocks are free, newest-admitted running request as the preemption victim.
+//
+// All output arrays are member vectors reused across steps (no allocation in
+// steady state once they have grown).
+#include <algorithm>
+#include <deque>
+#include <numeric>
+#include <vector>
+
+#include "bm_internal.hpp"
+#include "errors.hpp"
+
+using pagedkv::fail;
+
+struct pa_sched {
+  pa_bm* bm = nullptr;
+  int32_t n = 0;
+  int32_t max_blocks = 0;
+  std::vector<int32_t> arrival, prompt, output, generated;
+  std::vector<int32_t> arrival_order;
+  int32_t next_arrival = 0;
+  std::deque<int64_t> waiting;
+  std::vector<int64_t> running;
+  std::vector<char> is_running;
+  std::vector<int32_t> admit_len;
+  int32_t n_finished = 0;
+  int32_t step_idx = 0;
+  // step outputs
+  std::vector<int64_t> o_running, o_decode_slots, o_prompt_seqs, o_prompt_slots;
+  std::vector<int64_t> o_admitted, o_preempted, o_finished;
+  std::vector<int32_t> o_seq_lens, o_block_tables, o_prompt_lens, o_cow_src, o_cow_dst;
+  std::vector<int64_t> slot_of;  // per request: slot appended this step
+};
+
+namespace {
+
+void publish(pa_sched* s, pa_step_out* out) {
+  out->num_running = (int32_t)s->o_running.size();
+  out->max_blocks_per_seq = s->max_blocks;
+  out->running = s->o_running.data();
+  out->seq_lens = s->o_seq_lens.data();
+  out->block_tables = s->o_block_tables.data();
+  out->decode_slots = s->o_decode_slots.data();
+  out->num_prompt_seqs = (int32_t)s->o_prompt_seqs.size();
+  out->num_prompt_tokens = (int32_t)s->o_prompt_slots.size();
+  out->prompt_seqs = s->o_prompt_seqs.data();
+  out->prompt_lens = s->o_prompt_lens.data();
+  out->prompt_slots = s->o_prompt_slots.data();
+  out->num_cow = (int32_t)s->o_cow_src.size();
+  out->cow_src = s->o_cow_src.data();
+  out->cow_dst = s->o_cow_dst.data();
+  out->num_admitted = (int32_t)s->o_admitted.size();
+  out->admitted = s->o_admitted.data();
+  out->num_preempted = (int32_t)s->o_preempted.size();
+  out->preempted = s->o_preempted.data();
+  out->num_finished = (int32_t)s->o_finished.size();
+  out->finished = s->o_finished.data();
+  out->num_waiting = (int32_t)s->waiting.size();
+  out->num_free_blocks = s->bm->count;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_sched_create(pa_bm* bm, const int32_t* arrival_step, const int32_t* prompt_len,
+                          const int32_t* output_len, int32_t n_requests,
+                          int32_t max_blocks_per_seq, pa_sched** out) {
+  if (!out) return fail(PA_ERR_INVALID_ARG, "pa_sched_create: out is NULL");
+  *out = nullptr;
+  if (!bm || n_requests < 0 || max_blocks_per_seq <= 0 ||
+      (n_requests > 0 && (!arrival_step || !prompt_len || !output_len)))
+    return fail(PA_ERR_INVALID_ARG, "pa_sched_create: bad argument");
+  for (int32_t i = 0; i < n_requests; ++i) {
+    if (arrival_step[i] < 0 || prompt_len[i] < 1 || output_len[i] < 1)
+      return fail(PA_ERR_INVALID_ARG, "pa_sched_create: request %d (arrival %d, prompt %d, output %d)",
+                  i, arrival_step[i], prompt_len[i], output_len[i]);
+    if ((int64_t)prompt_len[i] + output_len[i] > (int64_t)max_blocks_per_seq * PA_BLOCK_SIZE)
+      return fail(PA_ERR_CAPACITY, "pa_sched_create: request %d needs more than %d blocks", i,
+                  max_blocks_per_seq);
+  }
+  pa_sched* s = new pa_sched();
+  s->bm = bm;
+  s->n = n_requests;
+  s->max_blocks = max_blocks_per_seq;
+  s->arrival.assign(arrival_step, arrival_step + n_requests);
+  s->prompt.assign(prompt_len, prompt_len + n_requests);
+  s->output.assign(output_len, output_len + n_requests);
+  s->generated.assign(n_requests, 0);
+  s->is_running.assign(n_requests, 0);
+  s->admit_len.assign(n_requests, 0);
+  s->slot_of.assign(n_requests, -1);
+  s->arrival_order.resize(n_requests);
+  std::iota(s->arrival_order.begin(), s->arrival_order.end(), 0);
+  std::stable_sort(s->arrival_order.begin(), s->arrival_order.end(),
+                   [s](int32_t a, int32_t b) { return s->arrival[a] < s->arrival[b]; });
+  *out = s;
+  return PA_OK;
+}
+
+void pa_sched_destroy(pa_sched* s) { delete s; }
+
+pa_status pa_sched_step(pa_sched* s, pa_step_out* out) {
+  if (!s || !out) return fail(PA_ERR_INVALID_ARG, "pa_sched_step: NULL argument");
+  pa_bm* bm = s->bm;
+  const int32_t step = s->step_idx++;
+  s->o_running.clear();
+  s->o_decode_slots.clear();
+  s->o_prompt_seqs.clear();
+  s->o_prompt_slots.clear();
+  s->o_admitted.clear();
+  s->o_preempted.clear();
+  s->o_finished.clear();
+  s->o_seq_lens.clear();
+  s->o_block_tables.clear();
+  s->o_prompt_lens.clear();
+  s->o_cow_src.clear();
+  s->o_cow_dst.clear();
+  out->step = step;
+
+  // 1. retire requests that generated all their tokens; pages return at once
+  {
+    size_t keep = 0;
+    for (size_t i = 0; i < s->running.size(); ++i) {
+      const int64_t r = s->running[i];
+      if (s->generated[r] >= s->output[r]) {
+        pa_status st = pa_bm_free(bm, r);
+        if (st != PA_OK) return st;
+        s->is_running[r] = 0;
+        s->o_finished.push_back(r);
+      } else {
+        s->running[keep++] = r;
+      }
+    }
+    s->running.resize(keep);
+    s->n_finished += (int32_t)s->o_finished.size();
+  }
+
+  // 2. arrivals join the waiting tail in (arrival step, id) order
+  while (s->next_arrival < s->n && s->arrival[s->arrival_order[s->next_arrival]] <= step) {
+    s->waiting.push_back(s->arrival_order[s->next_arrival]);
+    ++s->next_arrival;
+  }
+
+  // 3. admit from the head while its pages fit (first come, first served)
+  while (!s->waiting.empty()) {
+    const int64_t r = s->waiting.front();
+    const int32_t total = s->prompt[r] + s->generated[r];
+    if (pagedkv::blocks_for(total) > bm->count) {
+      if (s->running.empty())
+        return fail(PA_ERR_NO_BLOCKS, "pa_sched_step: request %lld can never fit (%d tokens, %d blocks)",
+                    (long long)r, total, bm->num_blocks);
+      break;
+    }
+    s->waiting.pop_front();
+    pa_status st = pa_bm_allocate(bm, r, total);
+    if (st != PA_OK) return st;
+    s->running.push_back(r);
+    s->is_running[r] = 1;
+    s->o_admitted.push_back(r);
+    s->admit_len[r] = total;
+  }
+
+  // 4. grow every running request by one slot; preempt the newest on shortage
+  for (size_t i = 0; i < s->running.size(); ++i) {
+    const int64_t r = s->running[i];
+    bool stop = false;
+    for (;;) {
+      int64_t slot;
+      int32_t cs, cd;
+      pa_status st = pa_bm_append_slot(bm, r, &slot, &cs, &cd);
+      if (st == PA_OK) {
+        s->slot_of[r] = slot;
+        if (cs >= 0) {
+          s->o_cow_src.push_back(cs);
+          s->o_cow_dst.push_back(cd);
+        }
+        break;
+      }
+      if (st != PA_ERR_NO_BLOCKS) return st;
+      const int64_t victim = s->running.back();
+      s->running.pop_back();
+      st = pa_bm_free(bm, victim);
+      if (st != PA_OK) return st;
+      s->is_running[victim] = 0;
+      s->waiting.push_front(victim);
+      s->o_preempted.push_back(victim);
+      if (victim == r) {
+        if (s->running.empty())
+          return fail(PA_ERR_NO_BLOCKS, "pa_sched_step: request %lld cannot grow alone", (long long)r);
+        stop = true;
+        break;
+      }
+    }
+    if (stop) break;
+  }
+
+  // 5. describe the step's device work
+  const size_t nr = s->running.size();
+  s->o_running.assign(s->running.begin(), s->running.end());
+  s->o_seq_lens.resize(nr);
+  s->o_decode_slots.resize(nr);
+  s->o_block_tables.resize(nr * (size_t)s->max_blocks);
+  if (nr) {
+    pa_status st = pa_bm_pack(bm, s->o_running.data(), (int32_t)nr, s->max_blocks,
+                              s->o_block_tables.data(), s->o_seq_lens.data(), nullptr);
+    if (st != PA_OK) return st;
+  }
+  for (size_t i = 0; i < nr; ++i) s->o_decode_slots[i] = s->slot_of[s->running[i]];
+  for (int64_t r : s->o_admitted) {
+    if (!s->is_running[r]) continue;  // admitted, then preempted in the same step
+    const int32_t n = s->admit_len[r];
+    s->o_prompt_seqs.push_back(r);
+    s->o_prompt_lens.push_back(n);
+    const size_t at = s->o_prompt_slots.size();
+    s->o_prompt_slots.resize(at + n);
+    pa_status st = pa_bm_slots(bm, r, 0, n, s->o_prompt_slots.data() + at);
+    if (st != PA_OK) return st;
+  }
+
+  // 6. every running request generated one token
+  for (int64_t r : s->running) s->generated[r] += 1;
+
+  out->done = (s->n_finished == s->n) ? 1 : 0;
+  publish(s, out);
+  return PA_OK;
+}
+
+}  // extern "C"

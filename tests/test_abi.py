@@ -1,0 +1,108 @@
+"""The C-ABI library loads and exports every entry point include/pagedkv.h
+declares; host-side argument checks reject bad input before any device work
+(these calls never reach the GPU, so they run without one)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_400_b200 import binding as bd
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "pagedkv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("pa_reshape_and_cache", "pa_decode", "pa_decode_workspace_size",
+                 "pa_copy_blocks", "pa_get_device_error", "pa_bm_create", "pa_sched_step"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = C.CDLL(bd.lib()._name)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert missing == []
+
+
+def test_status_strings():
+    for code in range(10):
+        s = bd.lib().pa_status_string(code)
+        assert s and s != b"unknown status"
+
+
+def pool(num_blocks=8, heads=2, dim=128, dtype=bd.PA_BF16, bs=16):
+    return bd.pa_pool_desc(num_blocks, heads, dim, bs, dtype)
+
+
+def test_decode_rejects_bad_arguments_on_host():
+    L = bd.lib()
+    p = pool()
+    vp = C.c_void_p(16)  # never dereferenced: rejected before use
+    cases = [
+        (pool(dim=96), 2, 1),     # unsupported head_dim
+        (pool(bs=32), 2, 1),      # block size must be 16
+        (pool(heads=3), 4, 1),    # H not a multiple of Hkv
+        (pool(heads=1), 17, 1),   # group of 17
+    ]
+    for desc, H, want in cases:
+        st = L.pa_decode(vp, vp, vp, vp, 4, vp, 1, H, 0.1, desc, None, 0, 16, None)
+        assert st in (1, 2), (desc.head_dim, H, st)
+    # max_seq_len beyond the table width
+    assert L.pa_decode(vp, vp, vp, vp, 1, vp, 1, 2, 0.1, p, None, 0, 17, None) == 1
+    # NaN scale
+    assert L.pa_decode(vp, vp, vp, vp, 4, vp, 1, 2, float("nan"), p, None, 0, 16, None) == 1
+    # long sequences need a workspace
+    assert L.pa_decode(vp, vp, vp, vp, 512, vp, 64, 2, 0.1, p, None, 0, 8192, None) == 9
+    # misaligned pointers
+    odd = C.c_void_p(18)
+    assert L.pa_decode(odd, vp, vp, vp, 4, vp, 1, 2, 0.1, p, None, 0, 16, None) == 1
+    assert b"aligned" in L.pa_last_error()
+    # empty batch is a no-op
+    assert L.pa_decode(None, None, None, None, 4, None, 0, 2, 0.1, p, None, 0, 16, None) == 0
+
+
+def test_append_and_copy_reject_bad_arguments_on_host():
+    L = bd.lib()
+    vp = C.c_void_p(16)
+    assert L.pa_reshape_and_cache(vp, vp, vp, vp, -1, pool(), None) == 1
+    assert L.pa_reshape_and_cache(None, None, None, None, 0, pool(), None) == 0
+    assert L.pa_reshape_and_cache(vp, vp, vp, vp, 3, pool(dtype=7), None) == 2
+    assert L.pa_copy_blocks(vp, vp, vp, -2, pool(), None) == 1
+    assert L.pa_copy_blocks(None, None, None, 0, pool(), None) == 0
+
+
+def test_workspace_size_is_deterministic_and_zero_for_one_partition():
+    p = pool(num_blocks=32768, heads=8)
+    assert bd.lib().pa_decode_workspace_size(256, 32, p, 8192) == \
+        bd.lib().pa_decode_workspace_size(256, 32, p, 8192) > 0
+    S = bd.lib().pa_decode_partition_tokens(256, 32, p, 8192)
+    assert S % 16 == 0 and S >= 128
+    # a bound within the smallest partition (128 tokens) needs no workspace
+    assert bd.lib().pa_decode_workspace_size(4, 2, pool(heads=2), 128) == 0
+    assert bd.lib().pa_decode_workspace_size(0, 2, p, 100) == 0
+
+
+def test_bm_errors_are_statuses():
+    bm = bd.BlockManager(4)
+    with pytest.raises(bd.PagedKVError) as e:
+        bm.allocate(0, 100)
+    assert e.value.status == "NO_BLOCKS" and bm.num_free() == 4
+    bm.allocate(0, 10)
+    with pytest.raises(bd.PagedKVError) as e:
+        bm.allocate(0, 1)
+    assert e.value.status == "SEQ_EXISTS"
+    with pytest.raises(bd.PagedKVError) as e:
+        bm.free(5)
+    assert e.value.status == "UNKNOWN_SEQ"
+    with pytest.raises(bd.PagedKVError):
+        bd.BlockManager(4, [0, 1, 1, 2])
+    with pytest.raises(bd.PagedKVError) as e:
+        bd._check("pa_bm_create", bd.lib().pa_bm_create(4, 32, None, C.byref(C.c_void_p())))
+    assert e.value.status == "UNSUPPORTED"
