@@ -47,6 +47,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=256,
+                    help="sequences per GPU (256 is the workload; smaller only for profiling captures)")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bounded oracle sample for cpu_baseline")
@@ -58,7 +60,7 @@ def workload_description(case):
     lens = np.asarray(case.info["seq_lens_after_append"])
     return {
         "workload": "gqa_llama3_8b_decode: 32 q / 8 kv heads, head_dim 128, bf16, block_size 16, "
-                    "batch 256, seq_lens lognormal(median 1000, sigma 0.8) clipped [16, 8192], "
+                    f"batch {len(case.batch)}, seq_lens lognormal(median 1000, sigma 0.8) clipped [16, 8192], "
                     "32768-block pool, random placement; step = cache append + split-KV decode",
         "global_batch": None,
         "seq_len_mean": float(lens.mean()),
@@ -253,7 +255,7 @@ def run_ours(args, rank, world, dist):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    case = wl.gqa_case(args.seed + rank)
+    case = wl.gqa_case(args.seed + rank, batch=args.batch)
     prep = prepare_decode_step(case)
     B, H, D = len(case.batch), case.num_heads, case.head_dim
     pool = case.make_pool(dev)

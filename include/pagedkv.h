@@ -63,6 +63,8 @@ typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
 #define PA_DEVERR_BLOCK   2u  /* decode/copy: block id outside [0, num_blocks) */
 #define PA_DEVERR_SEQLEN  4u  /* decode: seq_len < 0, > max_seq_len, or beyond
                                  max_blocks_per_seq * 16                     */
+#define PA_DEVERR_TIMEOUT 8u  /* decode: a wait for staged data gave up after
+                                 2 s (the kernel returned instead of hanging) */
 
 /*
  * The KV pool of one attention layer: one contiguous device buffer

@@ -23,7 +23,7 @@ STATUS_NAMES = {
     5: "UNKNOWN_SEQ", 6: "DEVICE_BOUNDS", 7: "SEQ_EXISTS", 8: "CAPACITY", 9: "WORKSPACE",
 }
 PA_F32, PA_BF16 = 0, 1
-PA_DEVERR_SLOT, PA_DEVERR_BLOCK, PA_DEVERR_SEQLEN = 1, 2, 4
+PA_DEVERR_SLOT, PA_DEVERR_BLOCK, PA_DEVERR_SEQLEN, PA_DEVERR_TIMEOUT = 1, 2, 4, 8
 BLOCK_SIZE = 16
 
 
