@@ -71,6 +71,22 @@ def workload_description(case):
     }
 
 
+def rank_case(seed: int, rank: int, batch: int):
+    """The batch a rank owns: an independent GQA decode batch (seed + rank)."""
+    from paged_kv_cache_400_b200 import workloads as wl
+    return wl.gqa_case(seed + rank, batch=batch)
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Largest value over all ranks (the job's time is its slowest rank's)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def algorithmic_bytes(case, prep, partitions_per_seq, max_partitions):
     """Bytes the step must move at minimum (the kernel's roofline traffic)."""
     elt = 2
@@ -255,7 +271,7 @@ def run_ours(args, rank, world, dist):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    case = wl.gqa_case(args.seed + rank, batch=args.batch)
+    case = rank_case(args.seed, rank, args.batch)
     prep = prepare_decode_step(case)
     B, H, D = len(case.batch), case.num_heads, case.head_dim
     pool = case.make_pool(dev)
@@ -306,10 +322,7 @@ def run_ours(args, rank, world, dist):
     decode_ms = [e[1].elapsed_time(e[2]) for e in ev]
     assert pk.pa_get_device_error() == 0
 
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
     ms_per_step = total_ms / K
     value = world * B / (ms_per_step / 1e3)
 
@@ -342,10 +355,7 @@ def run_ours(args, rank, world, dist):
         stream.synchronize()
     e1 = time.perf_counter()
     e2e_s = (e1 - e0) / E
-    if dist is not None:
-        t = torch.tensor([e2e_s], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
+    e2e_s = max_over_ranks(e2e_s, dist, dev)
 
     if rank != 0:
         return
