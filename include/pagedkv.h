@@ -159,6 +159,38 @@ pa_status pa_decode(void* out, const void* q, const void* kv_pool,
                     size_t workspace_bytes, int32_t max_seq_len, void* stream);
 
 /*
+ * Decode without a workspace argument, for callers that cannot allocate
+ * device memory. The pages have no counterpart: this is an integration
+ * variant of pa_decode, not part of the method.
+ * Some callers hand this library only their inputs and outputs and may not
+ * allocate on the device themselves: a plugin inside a host engine whose
+ * device memory is all owned by that engine's own pool, or a decode loop that
+ * must not call cudaMalloc / cudaFree between steps because those calls can
+ * synchronise the whole device and stall the other streams. For them the
+ * split-KV partial results live in one fixed device array inside the library,
+ * PA_DECODE_NOALLOC_SCRATCH_BYTES in size, created on every GPU that loads the
+ * library and held until the process exits.
+ * Same arguments, results and errors as pa_decode, minus the workspace. This
+ * call allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any
+ *    stream capture.
+ *  - A shape whose partial results need more than
+ *    PA_DECODE_NOALLOC_SCRATCH_BYTES (pa_decode_workspace_size) is rejected
+ *    with PA_ERR_WORKSPACE before anything is enqueued; use pa_decode then.
+ *  - Every call uses the same array and it keeps the last call's contents.
+ *    Nothing in it must start at zero (each partial result is written before
+ *    it is read), but two calls that overlap on the GPU (different streams,
+ *    no ordering between them) race on it and may return wrong results.
+ */
+#define PA_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20)  /* 32 MiB per device */
+pa_status pa_decode_noalloc(void* out, const void* q, const void* kv_pool,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* seq_lens, int32_t num_seqs, int32_t num_heads,
+                            float scale, pa_pool_desc pool, int32_t max_seq_len,
+                            void* stream);
+
+/*
  * Block copy for copy-on-write: for i in [0, n) in order,
  *     kv_pool[dst[i]] = kv_pool[src[i]]    (the whole block: K and V, all heads).
  * src, dst: device int32 [n]. Pairs must not overlap (no block is both a source

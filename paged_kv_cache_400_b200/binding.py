@@ -197,6 +197,29 @@ def pa_decode(out, q, kv_pool, block_tables, seq_lens, scale, max_seq_len, works
         int(max_seq_len), _stream(stream)))
 
 
+def pa_decode_noalloc(out, q, kv_pool, block_tables, seq_lens, scale, max_seq_len, stream=None):
+    """pa_decode without a workspace, for callers that cannot allocate device
+    memory: the split-KV partial results go to the library's fixed per-device
+    array (PA_DECODE_NOALLOC_SCRATCH_BYTES). Shapes that need more are rejected
+    (PagedKVError WORKSPACE). Calls overlapping on the GPU share that array and
+    race."""
+    fn = lib().pa_decode_noalloc
+    fn.restype = C.c_int32
+    fn.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_int32,
+                   C.c_int32, C.c_float, pa_pool_desc, C.c_int32, C.c_void_p]
+    desc = pool_desc(kv_pool)
+    B, H, D = q.shape
+    if out.shape != q.shape or D != desc.head_dim:
+        raise ValueError("q, out must be [num_seqs][num_heads][head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.shape != (B,):
+        raise ValueError("block_tables must be [num_seqs][max_blocks], seq_lens [num_seqs]")
+    _check("pa_decode_noalloc", fn(
+        _dev(out, "out", kv_pool.dtype), _dev(q, "q", kv_pool.dtype), _dev(kv_pool, "kv_pool"),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(seq_lens, "seq_lens", torch.int32), B, H, float(scale), desc, int(max_seq_len),
+        _stream(stream)))
+
+
 def pa_copy_blocks(kv_pool, src, dst, stream=None):
     desc = pool_desc(kv_pool)
     n = src.numel()

@@ -3,6 +3,7 @@
 // per-device error word without relocatable device code.
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "../host/errors.hpp"
 #include "append.cuh"
@@ -233,3 +234,59 @@ pa_status pa_get_device_error(uint32_t* flags, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// pa_decode_noalloc: decode for callers that cannot allocate device memory.
+// The split-KV partial results go to one fixed array in this file instead of
+// a caller-provided workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+// Scratch of pa_decode_noalloc. One per device, created when the module is
+// loaded on that device and kept until exit; shared by every call.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_DECODE_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device. In host code the
+// array's name is only a stand-in, never a device address: the address comes
+// from cudaGetSymbolAddress, once per device, with that device current.
+pa_status noalloc_scratch(void** ptr) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode_noalloc: device ordinal %d >= %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(PA_ERR_CUDA, "pa_decode_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* kv_pool,
+                                       const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                       const int32_t* seq_lens, int32_t num_seqs, int32_t num_heads,
+                                       float scale, pa_pool_desc pool, int32_t max_seq_len,
+                                       void* stream) {
+  const size_t need = pa_decode_workspace_size(num_seqs, num_heads, pool, max_seq_len);
+  if (need > PA_DECODE_NOALLOC_SCRATCH_BYTES)
+    return fail(PA_ERR_WORKSPACE,
+                "pa_decode_noalloc: this shape needs %zu bytes of split-KV scratch, the fixed array holds %u; "
+                "use pa_decode with a workspace",
+                need, (unsigned)PA_DECODE_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  pa_status s = noalloc_scratch(&scratch);
+  if (s != PA_OK) return s;
+  return pa_decode(out, q, kv_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads, scale,
+                   pool, scratch, PA_DECODE_NOALLOC_SCRATCH_BYTES, max_seq_len, stream);
+}
