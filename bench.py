@@ -47,6 +47,10 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--workload", choices=["gqa", "mha", "prefix", "trace"], default="gqa",
+                    help="gqa is the benchmark line; the others are extra measurements")
+    ap.add_argument("--trace-layers", type=int, default=32)
+    ap.add_argument("--trace-requests", type=int, default=2000)
     ap.add_argument("--batch", type=int, default=256,
                     help="sequences per GPU (256 is the workload; smaller only for profiling captures)")
     ap.add_argument("--e2e-steps", type=int, default=None)
@@ -56,12 +60,23 @@ def parse_args():
     return ap.parse_args()
 
 
-def workload_description(case):
-    lens = np.asarray(case.info["seq_lens_after_append"])
+WORKLOAD_TEXT = {
+    "gqa_llama3_8b": "gqa_llama3_8b_decode: 32 q / 8 kv heads, head_dim 128, bf16, block_size 16, "
+                     "batch {B}, seq_lens lognormal(median 1000, sigma 0.8) clipped [16, 8192], "
+                     "32768-block pool, random placement; step = cache append + split-KV decode",
+    "mha_llama2_7b": "mha_llama2_7b_decode: 32 q = 32 kv heads, head_dim 128, bf16, block_size 16, "
+                     "batch {B}, seq_lens uniform [128, 2048], 16384-block pool, random placement; "
+                     "step = cache append + split-KV decode",
+    "shared_prefix": "shared_prefix_decode: 32 seqs sharing a 1536-token prefix + suffixes U[0,512], "
+                     "8 prompts x 4 samples forking at a partial block (copy-on-write); 32/8 heads, "
+                     "head_dim 128, bf16, 4096-block pool; step = COW block copy + append + decode",
+}
+
+
+def workload_description(case, seq_lens):
+    lens = np.asarray(seq_lens)
     return {
-        "workload": "gqa_llama3_8b_decode: 32 q / 8 kv heads, head_dim 128, bf16, block_size 16, "
-                    f"batch {len(case.batch)}, seq_lens lognormal(median 1000, sigma 0.8) clipped [16, 8192], "
-                    "32768-block pool, random placement; step = cache append + split-KV decode",
+        "workload": WORKLOAD_TEXT[case.name].format(B=len(case.batch)),
         "global_batch": None,
         "seq_len_mean": float(lens.mean()),
         "seq_len_max": int(lens.max()),
@@ -71,9 +86,13 @@ def workload_description(case):
     }
 
 
-def rank_case(seed: int, rank: int, batch: int):
-    """The batch a rank owns: an independent GQA decode batch (seed + rank)."""
+def rank_case(seed: int, rank: int, batch: int, workload: str = "gqa"):
+    """The batch a rank owns: an independent decode batch (seed + rank)."""
     from paged_kv_cache_400_b200 import workloads as wl
+    if workload == "mha":
+        return wl.mha_case(seed + rank)
+    if workload == "prefix":
+        return wl.prefix_case(seed + rank)
     return wl.gqa_case(seed + rank, batch=batch)
 
 
@@ -164,10 +183,14 @@ class ClockSampler:
                 "samples": len(inside), "note": note}
 
 
+DECODE_KERNEL_SOURCES = ("common.cuh", "decode_common.cuh", "decode_staged.cuh", "ptx.cuh")
+
+
 def kernel_source_digest():
+    """Digest of the sources the staged decode kernel is compiled from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_400_b200", "csrc", "device")
-    for n in sorted(os.listdir(csrc)):
+    for n in DECODE_KERNEL_SOURCES:
         with open(os.path.join(csrc, n), "rb") as f:
             h.update(n.encode() + f.read())
     return h.hexdigest()[:16]
@@ -246,7 +269,7 @@ def run_reference(args, rank, world):
             times.append(dt)
     total = sum(times)
     value = per_step * len(times) / total
-    cfg = workload_description(case)
+    cfg = workload_description(case, ost.lens)
     cfg["global_batch"] = per_step
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
@@ -271,7 +294,7 @@ def run_ours(args, rank, world, dist):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    case = rank_case(args.seed, rank, args.batch)
+    case = rank_case(args.seed, rank, args.batch, args.workload)
     prep = prepare_decode_step(case)
     B, H, D = len(case.batch), case.num_heads, case.head_dim
     pool = case.make_pool(dev)
@@ -286,9 +309,17 @@ def run_ours(args, rank, world, dist):
     parts = [(int(n) + S - 1) // S for n in prep.seq_lens]
     nbytes = algorithmic_bytes(case, prep, parts, max(parts))
     stream = torch.cuda.current_stream()
+    cow_src = torch.from_numpy(prep.cow_src).to(dev) if len(prep.cow_src) else None
+    cow_dst = torch.from_numpy(prep.cow_dst).to(dev) if len(prep.cow_dst) else None
+
+    def append():
+        # the step's copy-on-write copies (shared-prefix workload) come first
+        if cow_src is not None:
+            pk.pa_copy_blocks(pool, cow_src, cow_dst)
+        pk.pa_reshape_and_cache(k, v, pool, slots)
 
     def step():
-        pk.pa_reshape_and_cache(k, v, pool, slots)
+        append()
         pk.pa_decode(out, q, pool, bt, sl, case.scale, case.max_seq_len, ws)
 
     for _ in range(max(args.warmup, 3)):
@@ -307,7 +338,7 @@ def run_ours(args, rank, world, dist):
     t_start.record(stream)
     for i in range(K):
         ev[i][0].record(stream)
-        pk.pa_reshape_and_cache(k, v, pool, slots)
+        append()
         ev[i][1].record(stream)
         pk.pa_decode(out, q, pool, bt, sl, case.scale, case.max_seq_len, ws)
         ev[i][2].record(stream)
@@ -364,7 +395,7 @@ def run_ours(args, rank, world, dist):
     achieved = nbytes["decode"] / (dec_avg_ms / 1e3) / 1e9
     traffic, traffic_src = recorded_traffic()
     kv_gbs = nbytes["kv"] / (ms_per_step / 1e3) / 1e9
-    cfg = workload_description(case)
+    cfg = workload_description(case, prep.seq_lens)
     cfg["global_batch"] = B * world
     cfg["parallelism"] = f"dp{world} independent replicas (no exchange step)"
     cfg["partition_tokens"] = S
@@ -381,7 +412,7 @@ def run_ours(args, rank, world, dist):
                      "traffic": traffic, "traffic_source": traffic_src,
                      "algorithmic_bytes_per_launch": nbytes["decode"],
                      "avg_launch_ms": dec_avg_ms, "append_avg_ms": sum(append_ms) / K},
-        "gpu_launches": K * (2 + (1 if max(parts) > 1 else 0)),
+        "gpu_launches": K * (2 + (1 if max(parts) > 1 else 0) + (1 if cow_src is not None else 0)),
         "clocks": sampler.summary(wall0, wall1),
         "e2e": {"value": world * B / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
@@ -395,6 +426,80 @@ def run_ours(args, rank, world, dist):
             "value": done / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"{done} of {B} sequences (random order), one decode token each: oracle "
                       f"gather through its own block tables + fp64 attention, {el:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
+def run_trace(args, rank, world):
+    """The 2000-request arrival trace through the C++ scheduler and the kernels:
+    per step, pa_sched_step, then for each of the layers the prompt append, the
+    decode-token append and paged decode. Inputs (the synthetic stand-in for the
+    model's K/V/Q projections) are generated on the device before each step's
+    layer loop and are outside every timed region. Reports generated tokens per
+    second of device time of the layer loops, and end to end (scheduler + index
+    copies + layer loops, wall clock, excluding input generation)."""
+    import torch
+
+    import paged_kv_cache_400_b200 as pk
+    from paged_kv_cache_400_b200 import workloads as wl
+    from paged_kv_cache_400_b200.engine import DecodeEngine
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    tr = wl.trace_case(args.seed + rank, n_requests=args.trace_requests, num_layers=args.trace_layers)
+    eng = DecodeEngine(tr.num_blocks, tr.num_layers, tr.num_heads, tr.num_kv_heads, tr.head_dim,
+                       tr.arrival_step, tr.prompt_len, tr.output_len, tr.table_width, tr.scale, dev)
+    stream = torch.cuda.current_stream()
+    events = []
+    tokens = kv_tokens = prompt_tokens = steps = preempted = 0
+    host_s = e2e_s = 0.0
+    sampler = ClockSampler(local)
+    sampler.start()
+    wall0 = time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        idx = eng.schedule()
+        t1 = time.perf_counter()
+        host_s += t1 - t0
+        n = len(idx.running)
+        if n:
+            reqs_p, pos_p = eng.prompt_positions(idx)
+            inputs = tr.step_inputs(idx.step, idx.running, idx.seq_lens, reqs_p, pos_p, dev)
+            torch.cuda.synchronize()
+            t2 = time.perf_counter()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            eng.run_layers(idx, inputs)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            e2e_s += (t1 - t0) + (time.perf_counter() - t2)
+            events.append((e0, e1))
+            tokens += n
+            kv_tokens += int(idx.seq_lens.astype(np.int64).sum())
+            prompt_tokens += len(idx.prompt_slots)
+        steps += 1
+        preempted += idx.record.preempted
+        if idx.done:
+            break
+    wall1 = time.perf_counter()
+    sampler.stop()
+    assert pk.pa_get_device_error() == 0
+    gpu_s = sum(a.elapsed_time(b) for a, b in events) / 1e3
+    eng.close()
+    kv_bytes = kv_tokens * 2 * tr.num_kv_heads * tr.head_dim * 2 * tr.num_layers
+    line = {
+        "workload": f"continuous-batching trace: {args.trace_requests} requests, Poisson(50) arrivals/step, "
+                    "prompts U[16,1024], outputs geometric mean 200 cap 2048, 40000-block pools, "
+                    f"{tr.num_layers} layers x (prompt append + decode-token append + paged decode), "
+                    "32/8 heads, head_dim 128, bf16",
+        "metric": "generated tokens/s (device time of the layer loops)", "value": tokens / gpu_s,
+        "unit": "tokens/s", "steps": steps, "generated_tokens": tokens, "prompt_tokens_written": prompt_tokens,
+        "preemptions": preempted, "gpu_s": gpu_s, "host_scheduler_s": host_s,
+        "kv_read_tb": kv_bytes / 1e12, "kv_read_gbs": kv_bytes / gpu_s / 1e9,
+        "e2e": {"value": tokens / e2e_s, "unit": "tokens/s",
+                "note": "pa_sched_step + index H2D + layer loops, wall clock; input generation excluded"},
+        "wall_s": wall1 - wall0, "clocks": sampler.summary(wall0, wall1),
+    }
     print(json.dumps(line), flush=True)
 
 
@@ -416,6 +521,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.workload == "trace":
+            run_trace(args, rank, world)
         else:
             run_ours(args, rank, world, dist)
     finally:

@@ -1,0 +1,154 @@
+"""Continuous-batching decode loop over per-layer paged KV pools.
+
+Each step the host scheduler (pa_sched_step, C++) decides which requests run,
+which are admitted (their prompt K/V are (re)written: recompute), which grow a
+block, which are preempted or finish; then, for every layer, the step's device
+work runs through the C ABI: copy-on-write block copies, the prompt-token
+append, the decode-token append, and paged decode over the running batch
+("vLLM 原理：PagedAttention 和 Continuous Batching" / "vLLM 的调度 / 调度流程";
+"大模型推理性能优化：PagedAttention与Continuous Batching原理与实践" §2.3).
+
+The model around attention is out of scope: the caller supplies the K/V of
+(layer, request, position) and the query of (layer, step, request), e.g. the
+seeded synthetic values of workloads.TraceCase.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+from . import binding as bd
+
+
+@dataclass
+class StepRecord:
+    step: int
+    num_running: int
+    num_prompt_tokens: int
+    admitted: int
+    preempted: int
+    finished: int
+    num_free_blocks: int
+    kernel_ms: float = 0.0     # device time of the layer loop (CUDA events)
+    host_ms: float = 0.0       # pa_sched_step + index packing
+
+
+@dataclass
+class StepIndices:
+    """Host copies of one step's index arrays (from pa_step_out)."""
+    step: int
+    running: np.ndarray
+    seq_lens: np.ndarray
+    block_tables: np.ndarray
+    decode_slots: np.ndarray
+    prompt_seqs: np.ndarray
+    prompt_lens: np.ndarray
+    prompt_slots: np.ndarray
+    cow_src: np.ndarray
+    cow_dst: np.ndarray
+    done: bool
+    record: StepRecord = field(default=None)
+
+
+class DecodeEngine:
+    def __init__(self, num_blocks, num_layers, num_heads, num_kv_heads, head_dim, arrival_step,
+                 prompt_len, output_len, table_width, scale, device, dtype=torch.bfloat16,
+                 max_seq_len=None):
+        self.device = torch.device(device)
+        self.num_layers = num_layers
+        self.num_heads = num_heads
+        self.num_kv_heads = num_kv_heads
+        self.head_dim = head_dim
+        self.scale = scale
+        self.table_width = table_width
+        self.max_seq_len = max_seq_len or table_width * bd.BLOCK_SIZE
+        self.bm = bd.BlockManager(num_blocks)
+        self.sched = bd.Scheduler(self.bm, arrival_step, prompt_len, output_len, table_width)
+        shape = (num_blocks, 2, num_kv_heads, bd.BLOCK_SIZE, head_dim)
+        self.pools = [torch.empty(shape, dtype=dtype, device=self.device) for _ in range(num_layers)]
+        self._ws = None
+        self._ws_batch = 0
+
+    def close(self):
+        self.sched.close()
+        self.bm.close()
+
+    # ---- host side -----------------------------------------------------------
+    def schedule(self) -> StepIndices:
+        import time
+        t0 = time.perf_counter()
+        o = self.sched.step_raw()
+        n = o.num_running
+
+        def arr(ptr, count, dt, shape=None):
+            if count == 0:
+                return np.empty(shape if shape else 0, dtype=dt)
+            a = np.ctypeslib.as_array(ptr, shape=(count,)).copy()
+            return a.reshape(shape) if shape else a
+
+        idx = StepIndices(
+            step=o.step,
+            running=arr(o.running, n, np.int64),
+            seq_lens=arr(o.seq_lens, n, np.int32),
+            block_tables=arr(o.block_tables, n * o.max_blocks_per_seq, np.int32,
+                             (n, o.max_blocks_per_seq)),
+            decode_slots=arr(o.decode_slots, n, np.int64),
+            prompt_seqs=arr(o.prompt_seqs, o.num_prompt_seqs, np.int64),
+            prompt_lens=arr(o.prompt_lens, o.num_prompt_seqs, np.int32),
+            prompt_slots=arr(o.prompt_slots, o.num_prompt_tokens, np.int64),
+            cow_src=arr(o.cow_src, o.num_cow, np.int32),
+            cow_dst=arr(o.cow_dst, o.num_cow, np.int32),
+            done=bool(o.done),
+        )
+        idx.record = StepRecord(o.step, n, o.num_prompt_tokens, o.num_admitted, o.num_preempted,
+                                o.num_finished, o.num_free_blocks,
+                                host_ms=1e3 * (time.perf_counter() - t0))
+        return idx
+
+    @staticmethod
+    def prompt_positions(idx: StepIndices):
+        """(request, position) of every prompt slot, in prompt_slots order."""
+        reqs = np.repeat(idx.prompt_seqs, idx.prompt_lens)
+        pos = np.concatenate([np.arange(n) for n in idx.prompt_lens]) if len(idx.prompt_lens) else \
+            np.empty(0, np.int64)
+        return reqs, pos
+
+    # ---- device side -------------------------------------------------------------
+    def workspace(self, batch):
+        if self._ws is None or batch > self._ws_batch:
+            self._ws = bd.alloc_workspace(batch, self.num_heads, self.pools[0], self.max_seq_len)
+            self._ws_batch = batch
+        return self._ws
+
+    def run_layers(self, idx: StepIndices, inputs, out=None):
+        """Device work of one step over all layers.
+
+        inputs: per layer l, a dict with "q" [n][H][D], "k_dec", "v_dec" [n][Hkv][D]
+        (the new token of each running request) and "k_prompt", "v_prompt"
+        [T][Hkv][D] (the prompt K/V in prompt_slots order), all on the device.
+        Returns the attention outputs per layer ([n][H][D] each)."""
+        dev = self.device
+        n = len(idx.running)
+        if n == 0:
+            return []
+        bt = torch.from_numpy(idx.block_tables).to(dev, non_blocking=True)
+        sl = torch.from_numpy(idx.seq_lens).to(dev, non_blocking=True)
+        ds = torch.from_numpy(idx.decode_slots).to(dev, non_blocking=True)
+        ps = torch.from_numpy(idx.prompt_slots).to(dev, non_blocking=True) if len(idx.prompt_slots) else None
+        cs = torch.from_numpy(idx.cow_src).to(dev) if len(idx.cow_src) else None
+        cd = torch.from_numpy(idx.cow_dst).to(dev) if len(idx.cow_dst) else None
+        ws = self.workspace(n)
+        outs = out if out is not None else [torch.empty(n, self.num_heads, self.head_dim,
+                                                         dtype=self.pools[0].dtype, device=dev)
+                                             for _ in range(self.num_layers)]
+        for l, pool in enumerate(self.pools):
+            x = inputs[l]
+            if cs is not None:
+                bd.pa_copy_blocks(pool, cs, cd)
+            if ps is not None:
+                bd.pa_reshape_and_cache(x["k_prompt"], x["v_prompt"], pool, ps)
+            bd.pa_reshape_and_cache(x["k_dec"], x["v_dec"], pool, ds)
+            bd.pa_decode(outs[l], x["q"], pool, bt, sl, self.scale, self.max_seq_len, ws)
+        return outs

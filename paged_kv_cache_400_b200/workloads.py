@@ -83,8 +83,9 @@ def stream_key(*coords: int) -> int:
     return _s64(k)
 
 
-def values(key: int, counters: torch.Tensor) -> torch.Tensor:
-    """Irwin-Hall(12) values (fp32) at the given int64 counters of stream `key`."""
+def values(key, counters: torch.Tensor) -> torch.Tensor:
+    """Irwin-Hall(12) values (fp32) at the given int64 counters of stream `key`
+    (an int, or an int64 tensor of keys broadcast against the counters)."""
     n = counters.to(torch.int64) * 2
     h1 = _mix(n * _GAMMA + key)
     h2 = _mix((n + 1) * _GAMMA + key)
@@ -305,6 +306,49 @@ class TraceCase:
         x = x.reshape(len(r), 2, self.num_kv_heads, self.head_dim)
         return x[:, 0].contiguous(), x[:, 1].contiguous()
 
+    def step_inputs(self, step: int, running, seq_lens, prompt_reqs, prompt_pos, device,
+                    chunk_elems: int = 1 << 26):
+        """Per-layer inputs of one continuous-batching step: the query and the
+        new token's K/V of each running request (position seq_len - 1), and the
+        prompt K/V of the (re)admitted requests, generated layer by layer in
+        chunks of at most `chunk_elems` values."""
+        per_tok = 2 * self.num_kv_heads * self.head_dim
+        reqs_p = np.asarray(prompt_reqs, np.int64)
+        pos_p = np.asarray(prompt_pos, np.int64)
+        dec_pos = np.asarray(seq_lens, np.int64) - 1
+        step_chunk = max(1, chunk_elems // per_tok)
+        dt = TORCH_DTYPE[self.dtype]
+        n = len(running)
+        L = self.num_layers
+        # decode-token K/V and queries of every layer in one generator call each
+        kv_keys = torch.tensor([stream_key(self.seed, TAG_TRACE_KV, l) for l in range(L)],
+                               dtype=torch.int64, device=device)[:, None]
+        q_keys = torch.tensor([stream_key(self.seed, TAG_TRACE_Q, l) for l in range(L)],
+                              dtype=torch.int64, device=device)[:, None]
+        r = torch.as_tensor(np.asarray(running, np.int64), device=device)
+        p = torch.as_tensor(dec_pos, device=device)
+        c = (((r * TRACE_MAX_POS + p) * per_tok)[:, None]
+             + torch.arange(per_tok, device=device)[None, :]).reshape(1, -1)
+        kv_all = values(kv_keys, c).to(dt).reshape(L, n, 2, self.num_kv_heads, self.head_dim)
+        per_q = self.num_heads * self.head_dim
+        cq = (((step * TRACE_MAX_REQ + r) * per_q)[:, None]
+              + torch.arange(per_q, device=device)[None, :]).reshape(1, -1)
+        q_all = values(q_keys, cq).to(dt).reshape(L, n, self.num_heads, self.head_dim)
+        out = []
+        for layer in range(L):
+            k_d = kv_all[layer, :, 0].contiguous()
+            v_d = kv_all[layer, :, 1].contiguous()
+            q = q_all[layer].contiguous()
+            if len(reqs_p) <= step_chunk:
+                k_p, v_p = self.kv_values(layer, reqs_p, pos_p, device)
+            else:
+                parts = [self.kv_values(layer, reqs_p[i:i + step_chunk], pos_p[i:i + step_chunk], device)
+                         for i in range(0, len(reqs_p), step_chunk)]
+                k_p = torch.cat([a for a, _ in parts])
+                v_p = torch.cat([b for _, b in parts])
+            out.append({"q": q, "k_dec": k_d, "v_dec": v_d, "k_prompt": k_p, "v_prompt": v_p})
+        return out
+
     def q_values(self, layer: int, step: int, reqs, device="cpu"):
         """Query of each request in `reqs` at (layer, step): [n][H][D]."""
         per = self.num_heads * self.head_dim
@@ -315,7 +359,7 @@ class TraceCase:
 
 
 def trace_case(seed: int = 0, n_requests: int = 2000, rate: float = 50.0,
-               num_blocks: int = 40000, num_layers: int = 32) -> TraceCase:
+               num_blocks: int = 40000, num_layers: int = 32, output_cap: int = 2048) -> TraceCase:
     rng = np.random.default_rng(seed + 505)
     arrivals = []
     step = 0
@@ -325,7 +369,7 @@ def trace_case(seed: int = 0, n_requests: int = 2000, rate: float = 50.0,
         step += 1
     arrivals = np.asarray(arrivals[:n_requests], dtype=np.int32)
     prompt = rng.integers(16, 1024, size=n_requests, endpoint=True).astype(np.int32)
-    output = np.minimum(rng.geometric(1.0 / 200.0, size=n_requests), 2048).astype(np.int32)
+    output = np.minimum(rng.geometric(1.0 / 200.0, size=n_requests), output_cap).astype(np.int32)
     return TraceCase(seed=seed, arrival_step=arrivals, prompt_len=prompt, output_len=output,
                      num_blocks=num_blocks, num_layers=num_layers, num_heads=32,
                      num_kv_heads=8, head_dim=128, dtype="bf16", scale=128 ** -0.5,

@@ -1,0 +1,92 @@
+"""GPU parity of the continuous-batching trace: the C++ scheduler drives the
+device loop (prompt append, decode-token append, paged decode per layer) over
+an arrival trace with preemptions; at sampled steps the fp64 oracle, with its
+own scheduler replay, block tables and pool built from the generator's K/V,
+must agree with the GPU attention output of every sampled request.
+
+The K/V of (layer, request, position) are a fixed function of those
+coordinates, so a request recomputed after preemption must see exactly the
+values it had before; any misplaced write in any earlier step shows up as an
+attention mismatch here.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as oa
+from oracle.block_manager import OracleBlockManager
+from oracle.scheduler import OracleScheduler
+from paged_kv_cache_400_b200 import workloads as wl
+from paged_kv_cache_400_b200.engine import DecodeEngine
+
+from oracle_side import storage_bits
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def layer_inputs(trace, eng, idx, layer, device):
+    reqs_p, pos_p = eng.prompt_positions(idx)
+    k_p, v_p = trace.kv_values(layer, reqs_p, pos_p, device)
+    k_d, v_d = trace.kv_values(layer, idx.running, idx.seq_lens.astype(np.int64) - 1, device)
+    q = trace.q_values(layer, idx.step, idx.running, device)
+    return {"q": q, "k_dec": k_d, "v_dec": v_d, "k_prompt": k_p, "v_prompt": v_p}
+
+
+def oracle_attention(trace, layer, step, req, table, length):
+    """Oracle: scatter the request's K/V (generator values) through its own
+    block table into a compact pool, then gather-and-attend in fp64."""
+    ids = sorted(set(table))
+    remap = {b: i for i, b in enumerate(ids)}
+    pool = np.zeros((len(ids), 2, trace.num_kv_heads, 16, trace.head_dim), dtype=np.uint16)
+    pos = np.arange(length)
+    k, v = trace.kv_values(layer, [req] * length, pos, "cpu")
+    slots = [remap[table[p // 16]] * 16 + p % 16 for p in range(length)]
+    assert oa.reshape_and_cache(pool, storage_bits(k), storage_bits(v), slots) == []
+    q = storage_bits(trace.q_values(layer, step, [req], "cpu"))
+    tab = [[remap[b] for b in table]]
+    return oa.paged_decode(q, pool, tab, [length], trace.scale, "bf16")[0]
+
+
+def test_trace_with_preemption_matches_oracle():
+    trace = wl.trace_case(seed=5, n_requests=240, rate=16.0, num_blocks=1800, num_layers=2,
+                          output_cap=300)
+    eng = DecodeEngine(trace.num_blocks, trace.num_layers, trace.num_heads, trace.num_kv_heads,
+                       trace.head_dim, trace.arrival_step, trace.prompt_len, trace.output_len,
+                       trace.table_width, trace.scale, DEV)
+    obm = OracleBlockManager(trace.num_blocks)
+    osch = OracleScheduler(obm, trace.arrival_step, trace.prompt_len, trace.output_len, trace.table_width)
+    rng = np.random.default_rng(0)
+    checked = preempted_seen = steps = 0
+    max_err = 0.0
+    while True:
+        idx = eng.schedule()
+        o = osch.step()
+        assert idx.running.tolist() == o["running"]
+        assert idx.decode_slots.tolist() == o["decode_slots"]
+        assert idx.prompt_slots.tolist() == o["prompt_slots"]
+        preempted_seen += len(o["preempted"])
+        steps += 1
+        if len(idx.running):
+            inputs = [layer_inputs(trace, eng, idx, l, DEV) for l in range(trace.num_layers)]
+            outs = eng.run_layers(idx, inputs)
+            sample_step = checked < 40 and ((idx.step % 20 == 0) or
+                                            (len(o["preempted"]) and idx.step % 3 == 0))
+            if sample_step:
+                layer = int(rng.integers(0, trace.num_layers))
+                rows = rng.choice(len(idx.running), size=min(3, len(idx.running)), replace=False)
+                got = outs[layer].float().cpu().numpy()
+                for i in rows:
+                    r = int(idx.running[i])
+                    ref = oracle_attention(trace, layer, idx.step, r, o["block_tables"][i][
+                        :(o["seq_lens"][i] + 15) // 16], o["seq_lens"][i])
+                    err = float(np.abs(got[i] - ref).max())
+                    max_err = max(max_err, err)
+                    assert err <= 1e-2, (idx.step, r, err)
+                    checked += 1
+        if idx.done:
+            break
+    import paged_kv_cache_400_b200 as pk
+    assert pk.pa_get_device_error() == 0
+    assert preempted_seen > 0 and checked >= 20, (preempted_seen, checked, steps)
+    eng.close()
