@@ -284,11 +284,28 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def timed_loop(K, stream, phases):
+    """Runs K steps; each step runs the callables of `phases` in order, with a
+    CUDA event between phases. Returns (total ms, per-phase ms lists)."""
+    import torch
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(phases) + 1)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        for j, fn in enumerate(phases):
+            fn()
+            ev[i][j + 1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    per = [[e[j].elapsed_time(e[j + 1]) for e in ev] for j in range(len(phases))]
+    return t0.elapsed_time(t1), per
+
+
 def run_ours(args, rank, world, dist):
     import torch
 
     import paged_kv_cache_400_b200 as pk
-    from paged_kv_cache_400_b200 import workloads as wl
     from paged_kv_cache_400_b200.scenario import prepare_decode_step
 
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -312,48 +329,46 @@ def run_ours(args, rank, world, dist):
     cow_src = torch.from_numpy(prep.cow_src).to(dev) if len(prep.cow_src) else None
     cow_dst = torch.from_numpy(prep.cow_dst).to(dev) if len(prep.cow_dst) else None
 
-    def append():
+    def cow():
         # the step's copy-on-write copies (shared-prefix workload) come first
         if cow_src is not None:
             pk.pa_copy_blocks(pool, cow_src, cow_dst)
+
+    def append_decode():   # the step as one call: append folded into decode
+        pk.pa_append_decode(out, q, k, v, pool, slots, bt, sl, case.scale, case.max_seq_len, ws)
+
+    def append():
         pk.pa_reshape_and_cache(k, v, pool, slots)
 
-    def step():
-        append()
+    def decode():
         pk.pa_decode(out, q, pool, bt, sl, case.scale, case.max_seq_len, ws)
 
     for _ in range(max(args.warmup, 3)):
-        step()
+        cow()
+        append_decode()
+        cow()
+        append()
+        decode()
     assert pk.pa_get_device_error() == 0
 
+    K = args.steps
     sampler = ClockSampler(local)
     sampler.start()
-    K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
-    t_start.record(stream)
-    for i in range(K):
-        ev[i][0].record(stream)
-        append()
-        ev[i][1].record(stream)
-        pk.pa_decode(out, q, pool, bt, sl, case.scale, case.max_seq_len, ws)
-        ev[i][2].record(stream)
-    t_end.record(stream)
-    torch.cuda.synchronize()
+    total_ms, (cow_ms, step_ms) = timed_loop(K, stream, [cow, append_decode])
     wall1 = time.perf_counter()
     if dist is not None:
         dist.barrier()
     sampler.stop()
-    total_ms = t_start.elapsed_time(t_end)
-    append_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    decode_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    # the same step as separate calls, for comparison
+    total_sep, (_, app_ms, dec_ms) = timed_loop(K, stream, [cow, append, decode])
     assert pk.pa_get_device_error() == 0
 
     total_ms = max_over_ranks(total_ms, dist, dev)
+    total_sep = max_over_ranks(total_sep, dist, dev)
     ms_per_step = total_ms / K
     value = world * B / (ms_per_step / 1e3)
 
@@ -381,24 +396,28 @@ def run_ours(args, rank, world, dist):
         slots.copy_(h_slots, non_blocking=True)
         bt.copy_(h_bt, non_blocking=True)
         sl.copy_(h_sl, non_blocking=True)
-        step()
+        cow()
+        append_decode()
         h_out.copy_(out, non_blocking=True)
         stream.synchronize()
     e1 = time.perf_counter()
-    e2e_s = (e1 - e0) / E
-    e2e_s = max_over_ranks(e2e_s, dist, dev)
+    e2e_s = max_over_ranks((e1 - e0) / E, dist, dev)
 
     if rank != 0:
         return
     peak, peak_src = measured_peak()
-    dec_avg_ms = sum(decode_ms) / K
-    achieved = nbytes["decode"] / (dec_avg_ms / 1e3) / 1e9
+    step_avg = sum(step_ms) / K
+    fused_bytes = nbytes["decode"] + nbytes["append"]
+    achieved = fused_bytes / (step_avg / 1e3) / 1e9
     traffic, traffic_src = recorded_traffic()
     kv_gbs = nbytes["kv"] / (ms_per_step / 1e3) / 1e9
     cfg = workload_description(case, prep.seq_lens)
     cfg["global_batch"] = B * world
     cfg["parallelism"] = f"dp{world} independent replicas (no exchange step)"
     cfg["partition_tokens"] = S
+    cfg["step"] = ("pa_append_decode (cache append folded into the split-KV decode kernel)"
+                   + (" after pa_copy_blocks" if cow_src is not None else ""))
+    dec_avg = sum(dec_ms) / K
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -406,26 +425,37 @@ def run_ours(args, rank, world, dist):
         "config": cfg,
         "kv_read_gbs": kv_gbs, "kv_frac_of_8tbs": kv_gbs / NOMINAL_HBM_GBS,
         "kv_frac_of_measured": kv_gbs / peak,
-        "roofline": {"kernel": "pa_decode (split-KV partition kernel + partition reduce)",
+        "roofline": {"kernel": "decode_staged_kernel with fused append (pa_append_decode; partition "
+                               "reduce launch included)",
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_src,
                      "traffic": traffic, "traffic_source": traffic_src,
-                     "algorithmic_bytes_per_launch": nbytes["decode"],
-                     "avg_launch_ms": dec_avg_ms, "append_avg_ms": sum(append_ms) / K},
-        "gpu_launches": K * (2 + (1 if max(parts) > 1 else 0) + (1 if cow_src is not None else 0)),
+                     "algorithmic_bytes_per_launch": fused_bytes, "avg_launch_ms": step_avg},
+        "separate_calls": {"ms_per_step": total_sep / K, "append_avg_ms": sum(app_ms) / K,
+                           "decode_avg_ms": dec_avg,
+                           "decode_frac_of_measured": nbytes["decode"] / (dec_avg / 1e3) / 1e9 / peak,
+                           "value": world * B / (total_sep / K / 1e3)},
+        "gpu_launches": K * (1 + (1 if max(parts) > 1 else 0) + (1 if cow_src is not None else 0)),
         "clocks": sampler.summary(wall0, wall1),
         "e2e": {"value": world * B / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "note": "per step: host table packing (pa_bm_pack), H2D of q/k/v/slots/tables/lens "
-                        "from pinned memory, append + decode, D2H of out, stream sync"},
+                        "from pinned memory, pa_append_decode, D2H of out, stream sync"},
         "library": os.path.relpath(pk.library_path(), ROOT),
     }
+    if case.name == "shared_prefix":
+        uniq = len({int(x) for row, n in zip(prep.block_tables, prep.seq_lens)
+                    for x in row[:(int(n) + 15) // 16]})
+        ub = uniq * 2 * case.num_kv_heads * 16 * D * 2
+        line["unique_kv_bytes"] = ub
+        line["unique_kv_gbs"] = ub / (ms_per_step / 1e3) / 1e9
     if not args.no_cpu_baseline and world == 1:
         done, el = oracle_sample(case, args.cpu_seconds)
         line["cpu_baseline"] = {
             "value": done / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"{done} of {B} sequences (random order), one decode token each: oracle "
-                      f"gather through its own block tables + fp64 attention, {el:.1f} s"}
+                      f"copy-on-write + append + gather through its own block tables + fp64 "
+                      f"attention, {el:.1f} s of oracle time"}
     print(json.dumps(line), flush=True)
 
 

@@ -159,6 +159,32 @@ pa_status pa_decode(void* out, const void* q, const void* kv_pool,
                     size_t workspace_bytes, int32_t max_seq_len, void* stream);
 
 /*
+ * One decode step in one call: the new token of every sequence is appended
+ * and attention runs over the updated cache. Same results, pool contents and
+ * errors as
+ *     pa_reshape_and_cache(k_new, v_new, kv_pool, slot_mapping, num_seqs, ...)
+ *     pa_decode(out, q, kv_pool, block_tables, ..., seq_lens, ...)
+ * when token b is sequence b's newest token, i.e. slot_mapping[b] is the slot
+ * of position seq_lens[b]-1 through block_tables[b] (or negative: not
+ * appended). For bf16 pools with head_dim 128 the append is folded into the
+ * decode kernel (no separate launch): the CTA that stages the block holding
+ * position seq_lens[b]-1 writes the new K/V row into that staged block and
+ * stores it to the pool. A token whose slot is not that position's slot is not
+ * written and raises PA_DEVERR_SLOT; a sequence of length 0 appends nothing.
+ * Other dtypes and head sizes run the two calls in sequence.
+ * k_new, v_new: device [num_seqs][num_kv_heads][head_dim], pool dtype, 16-byte
+ * aligned; slot_mapping: device int64 [num_seqs]. The remaining arguments are
+ * pa_decode's. The append/decode pairing of one step is the same as in the
+ * pages' step loop ([B] "vLLM 的调度 / 调度流程": run the step, append the token).
+ */
+pa_status pa_append_decode(void* out, const void* q, const void* k_new, const void* v_new,
+                           void* kv_pool, const int64_t* slot_mapping,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* seq_lens, int32_t num_seqs, int32_t num_heads,
+                           float scale, pa_pool_desc pool, void* workspace,
+                           size_t workspace_bytes, int32_t max_seq_len, void* stream);
+
+/*
  * Decode without a workspace argument, for callers that cannot allocate
  * device memory. The pages have no counterpart: this is an integration
  * variant of pa_decode, not part of the method.

@@ -70,6 +70,8 @@ def _declare(lib):
         "pa_decode_partition_tokens": (i32, [i32, i32, pa_pool_desc, i32]),
         "pa_decode": (i32, [vp, vp, vp, vp, i32, vp, i32, i32, f32, pa_pool_desc, vp, sz, i32, vp]),
         "pa_copy_blocks": (i32, [vp, vp, vp, i32, pa_pool_desc, vp]),
+        "pa_append_decode": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, f32, pa_pool_desc, vp, sz,
+                                   i32, vp]),
         "pa_get_device_error": (i32, [C.POINTER(C.c_uint32), vp]),
         "pa_status_string": (C.c_char_p, [i32]),
         "pa_last_error": (C.c_char_p, []),
@@ -195,6 +197,30 @@ def pa_decode(out, q, kv_pool, block_tables, seq_lens, scale, max_seq_len, works
         _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
         _dev(seq_lens, "seq_lens", torch.int32), B, H, float(scale), desc, ws_ptr, ws_bytes,
         int(max_seq_len), _stream(stream)))
+
+
+def pa_append_decode(out, q, k_new, v_new, kv_pool, slot_mapping, block_tables, seq_lens, scale,
+                     max_seq_len, workspace=None, stream=None):
+    """pa_reshape_and_cache of each sequence's new token followed by pa_decode,
+    in one call (one kernel for bf16 / head_dim 128)."""
+    desc = pool_desc(kv_pool)
+    B, H, D = q.shape
+    if out.shape != q.shape or D != desc.head_dim:
+        raise ValueError("q, out must be [num_seqs][num_heads][head_dim]")
+    if k_new.shape != (B, desc.num_kv_heads, D) or v_new.shape != k_new.shape:
+        raise ValueError("k_new, v_new must be [num_seqs][num_kv_heads][head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.shape != (B,) \
+            or slot_mapping.shape != (B,):
+        raise ValueError("block_tables [num_seqs][max_blocks], seq_lens and slot_mapping [num_seqs]")
+    ws_ptr, ws_bytes = C.c_void_p(0), 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    _check("pa_append_decode", lib().pa_append_decode(
+        _dev(out, "out", kv_pool.dtype), _dev(q, "q", kv_pool.dtype), _dev(k_new, "k_new", kv_pool.dtype),
+        _dev(v_new, "v_new", kv_pool.dtype), _dev(kv_pool, "kv_pool"),
+        _dev(slot_mapping, "slot_mapping", torch.int64), _dev(block_tables, "block_tables", torch.int32),
+        block_tables.shape[1], _dev(seq_lens, "seq_lens", torch.int32), B, H, float(scale), desc, ws_ptr,
+        ws_bytes, int(max_seq_len), _stream(stream)))
 
 
 def pa_decode_noalloc(out, q, kv_pool, block_tables, seq_lens, scale, max_seq_len, stream=None):

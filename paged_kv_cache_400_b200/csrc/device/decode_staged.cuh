@@ -19,7 +19,8 @@
 // warp keeps an online-softmax state (running max m, partial sum l, output
 // accumulator) in the log2 domain; the four states are merged through shared
 // memory at the end and either written out (one partition) or stored as a
-// partition state for the reduce kernel.
+// partition state for the merge kernel (partition_merge_kernel, launched as a
+// programmatic dependent so its launch overlaps this kernel's tail).
 //
 // Compute per block of 16 tokens:
 //  * head group G >= 2 (GQA): the group's query heads are the M dimension of
@@ -61,7 +62,7 @@ __device__ __forceinline__ uint32_t tile_chunk(int kv, int token, int chunk16) {
   return (uint32_t)((chunk16 >> 3) * 4096 + kv * 2048 + token * 128 + (((chunk16 & 7) ^ (token & 7)) << 4));
 }
 
-template <bool kMMA>
+template <bool kMMA, bool kAppend>
 __global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constant__ CUtensorMap tmap,
                                                             DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -78,6 +79,9 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constan
   const int32_t G = p.group;
   const int32_t H = p.num_heads;
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+  // the partition merge may be scheduled as soon as every CTA has started; it
+  // waits for this grid's completion before reading any partition state
+  grid_dependents_launch();
 
   const int32_t L = checked_len(p, b, part == 0 && g == 0 && threadIdx.x == 0);
   const int32_t S = p.partition_tokens;
@@ -105,13 +109,30 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constan
   }
   __syncwarp();
 
+  // Block ids of this warp's blocks, read once: lane i holds the id of the
+  // warp's i-th block (partition block warp + 4i), so issuing a load never
+  // waits on a table read.
+  const int32_t my_blk = lane < my ? __ldg(table + warp + lane * kStagedWarps) : -1;
+
+  // Fused append: the warp that will stage the block holding position L-1
+  // fetches the new token's K/V row (lanes 0-15: K chunks, 16-31: V chunks)
+  // and slot now, so the loads overlap the pipeline.
+  const bool app_here = kAppend && t1 == L && ((nb - 1) % kStagedWarps) == warp;
+  const int32_t app_iter = (nb - 1) / kStagedWarps;
+  uint4 app_val = make_uint4(0, 0, 0, 0);
+  int64_t app_slot = -1;
+  if (app_here) {
+    app_slot = __ldg(p.slot_mapping + b);
+    app_val = __ldg(reinterpret_cast<const uint4*>((lane >> 4) ? p.v_new : p.k_new) +
+                    ((size_t)b * p.num_kv_heads + g) * 16 + (lane & 15));
+  }
+
   uint32_t valid_mask = 0;  // bit s: stage s holds a real block
   auto issue = [&](int32_t i) {
     const int32_t s = i % kStagedStages;
-    const int32_t j = warp + i * kStagedWarps;
+    const int32_t blk = __shfl_sync(0xffffffffu, my_blk, i);
     int32_t ok = 0;
     if (lane == 0) {
-      const int32_t blk = __ldg(table + j);
       uint64_t* bar = &bars[warp][s];
       if (blk >= 0 && blk < p.num_blocks) {
         fence_proxy_async_smem();
@@ -130,6 +151,10 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constan
 
   const int32_t gid = lane >> 2;  // mma row group
   const int32_t tig = lane & 3;   // thread in group
+
+  // first loads in flight before anything else is read
+  const int32_t npre = my < kStagedStages ? my : kStagedStages;
+  for (int32_t i = 0; i < npre; ++i) issue(i);
 
   // ---- per-warp softmax state ---------------------------------------------
   // MMA: rows gid and gid+8 of the 16-row head tile.
@@ -173,8 +198,6 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constan
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
   }
 
-  const int32_t npre = my < kStagedStages ? my : kStagedStages;
-  for (int32_t i = 0; i < npre; ++i) issue(i);
 
   for (int32_t i = 0; i < my; ++i) {
     const int32_t s = i % kStagedStages;
@@ -192,6 +215,28 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constan
         *reinterpret_cast<uint4*>(wsm + s * kStageBytes + tile_chunk(1, row, e & 15)) = make_uint4(0, 0, 0, 0);
       }
       __syncwarp();
+    }
+    if constexpr (kAppend) {
+      // Fused cache append: this block holds position L-1, the step's new
+      // token. Its K/V row (this KV head) is written into the staged block and
+      // stored to the pool at the token's slot, which must be that position's
+      // slot through the table; otherwise PA_DEVERR_SLOT and nothing is written.
+      if (app_here && i == app_iter) {
+        const int32_t blk = __shfl_sync(0xffffffffu, my_blk, i);
+        const int32_t row = nvalid - 1;
+        if (app_slot >= 0) {
+          if (valid && app_slot == (int64_t)blk * 16 + row) {
+            const int32_t kv = lane >> 4;
+            const int32_t c = lane & 15;
+            *reinterpret_cast<uint4*>(wsm + s * kStageBytes + tile_chunk(kv, row, c)) = app_val;
+            uint4* pool = reinterpret_cast<uint4*>(const_cast<void*>(p.pool));
+            pool[(((size_t)blk * 2 + kv) * p.num_kv_heads + g) * 256 + row * 16 + c] = app_val;
+            __syncwarp();
+          } else if (lane == 0) {
+            raise_device_error(PA_DEVERR_SLOT);
+          }
+        }
+      }
     }
 
     if constexpr (kMMA) {
@@ -409,9 +454,9 @@ inline pa_status encode_pool_map(const DecodeParams& p, CUtensorMap* map) {
   return PA_OK;
 }
 
-template <bool kMMA>
+template <bool kMMA, bool kAppend>
 inline pa_status prepare_staged() {
-  static cudaError_t e = cudaFuncSetAttribute(decode_staged_kernel<kMMA>,
+  static cudaError_t e = cudaFuncSetAttribute(decode_staged_kernel<kMMA, kAppend>,
                                               cudaFuncAttributeMaxDynamicSharedMemorySize, kStagedSmem);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode: %s", cudaGetErrorString(e));
   return PA_OK;
@@ -422,19 +467,25 @@ inline pa_status launch_staged_bf16_d128(const DecodeParams& p, cudaStream_t st)
   pa_status s = encode_pool_map(p, &map);
   if (s != PA_OK) return s;
   dim3 grid(p.max_partitions, p.num_kv_heads, p.num_seqs);
-  if (p.group == 1) {
-    if ((s = prepare_staged<false>()) != PA_OK) return s;
-    decode_staged_kernel<false><<<grid, 128, kStagedSmem, st>>>(map, p);
+  const bool append = p.k_new != nullptr;
+  if (p.group == 1 && !append) {
+    if ((s = prepare_staged<false, false>()) != PA_OK) return s;
+    decode_staged_kernel<false, false><<<grid, 128, kStagedSmem, st>>>(map, p);
+  } else if (p.group == 1) {
+    if ((s = prepare_staged<false, true>()) != PA_OK) return s;
+    decode_staged_kernel<false, true><<<grid, 128, kStagedSmem, st>>>(map, p);
+  } else if (!append) {
+    if ((s = prepare_staged<true, false>()) != PA_OK) return s;
+    decode_staged_kernel<true, false><<<grid, 128, kStagedSmem, st>>>(map, p);
   } else {
-    if ((s = prepare_staged<true>()) != PA_OK) return s;
-    decode_staged_kernel<true><<<grid, 128, kStagedSmem, st>>>(map, p);
+    if ((s = prepare_staged<true, true>()) != PA_OK) return s;
+    decode_staged_kernel<true, true><<<grid, 128, kStagedSmem, st>>>(map, p);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode: launch failed: %s", cudaGetErrorString(e));
   if (p.max_partitions <= 1) return PA_OK;
-  partition_reduce_kernel<__nv_bfloat16, 128><<<dim3(p.num_heads, p.num_seqs), 128, 0, st>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode (reduce): launch failed: %s", cudaGetErrorString(e));
+  e = launch_partition_merge<__nv_bfloat16, 128>(p, st);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode (merge): launch failed: %s", cudaGetErrorString(e));
   return PA_OK;
 }
 

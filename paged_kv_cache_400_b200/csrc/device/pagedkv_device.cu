@@ -79,8 +79,9 @@ pa_status launch_generic(const pagedkv::DecodeParams& p, cudaStream_t st) {
   else pagedkv::decode_generic_kernel<T, D, 16><<<grid, 128, 0, st>>>(p);
   pa_status s = launch_status("pa_decode");
   if (s != PA_OK || p.max_partitions <= 1) return s;
-  pagedkv::partition_reduce_kernel<T, D><<<dim3(p.num_heads, p.num_seqs), D, 0, st>>>(p);
-  return launch_status("pa_decode (reduce)");
+  cudaError_t e = pagedkv::launch_partition_merge<T, D>(p, st);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode (merge): launch failed: %s", cudaGetErrorString(e));
+  return PA_OK;
 }
 
 }  // namespace
@@ -180,6 +181,9 @@ pa_status pa_decode(void* out, const void* q, const void* kv_pool, const int32_t
   p.seq_lens = seq_lens;
   p.ws_acc = reinterpret_cast<float*>(workspace);
   p.ws_ml = w.total ? reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + w.ml_offset) : nullptr;
+  p.k_new = nullptr;
+  p.v_new = nullptr;
+  p.slot_mapping = nullptr;
   p.max_blocks = max_blocks_per_seq;
   p.num_seqs = num_seqs;
   p.num_heads = num_heads;
@@ -201,6 +205,74 @@ pa_status pa_decode(void* out, const void* q, const void* kv_pool, const int32_t
                                 : launch_generic<__nv_bfloat16, 64>(p, st);
   }
   return pool.head_dim == 128 ? launch_generic<float, 128>(p, st) : launch_generic<float, 64>(p, st);
+}
+
+pa_status pa_append_decode(void* out, const void* q, const void* k_new, const void* v_new, void* kv_pool,
+                           const int64_t* slot_mapping, const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* seq_lens, int32_t num_seqs, int32_t num_heads, float scale,
+                           pa_pool_desc pool, void* workspace, size_t workspace_bytes, int32_t max_seq_len,
+                           void* stream) {
+  if (num_seqs > 0 && (!k_new || !v_new || !slot_mapping))
+    return fail(PA_ERR_INVALID_ARG, "pa_append_decode: NULL k_new, v_new or slot_mapping");
+  if (num_seqs > 0 && (!aligned16(k_new) || !aligned16(v_new)))
+    return fail(PA_ERR_INVALID_ARG, "pa_append_decode: k_new and v_new must be 16-byte aligned");
+  const bool staged = pool.dtype == PA_BF16 && pool.head_dim == 128 && pool.block_size == PA_BLOCK_SIZE;
+  if (!staged) {
+    // other shapes: the two calls in sequence (same results)
+    pa_status s = pa_reshape_and_cache(k_new, v_new, kv_pool, slot_mapping, num_seqs, pool, stream);
+    if (s != PA_OK) return s;
+    return pa_decode(out, q, kv_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads, scale, pool,
+                     workspace, workspace_bytes, max_seq_len, stream);
+  }
+  // Validate exactly as pa_decode does, then launch the decode kernel with the
+  // append folded in.
+  pa_status s = check_pool(pool, "pa_append_decode");
+  if (s != PA_OK) return s;
+  if (num_seqs < 0 || num_heads <= 0 || max_blocks_per_seq <= 0 || max_seq_len < 0)
+    return fail(PA_ERR_INVALID_ARG, "pa_append_decode: num_seqs %d, num_heads %d, max_blocks %d, max_seq_len %d",
+                num_seqs, num_heads, max_blocks_per_seq, max_seq_len);
+  if (num_heads % pool.num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "pa_append_decode: num_heads %d not a multiple of num_kv_heads %d", num_heads,
+                pool.num_kv_heads);
+  const int32_t G = num_heads / pool.num_kv_heads;
+  if (G > 16) return fail(PA_ERR_UNSUPPORTED, "pa_append_decode: head group %d > 16", G);
+  if (num_seqs > 65535) return fail(PA_ERR_UNSUPPORTED, "pa_append_decode: num_seqs %d > 65535", num_seqs);
+  if ((int64_t)max_seq_len > (int64_t)max_blocks_per_seq * PA_BLOCK_SIZE)
+    return fail(PA_ERR_INVALID_ARG, "pa_append_decode: max_seq_len %d > max_blocks_per_seq * 16", max_seq_len);
+  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "pa_append_decode: scale is not finite");
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !kv_pool || !block_tables || !seq_lens)
+    return fail(PA_ERR_INVALID_ARG, "pa_append_decode: NULL pointer");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(kv_pool))
+    return fail(PA_ERR_INVALID_ARG, "pa_append_decode: out, q and kv_pool must be 16-byte aligned");
+  const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, pool, max_seq_len > 0 ? max_seq_len : 1);
+  if (w.total > 0 && (!workspace || workspace_bytes < w.total))
+    return fail(PA_ERR_WORKSPACE, "pa_append_decode: workspace %zu bytes at %p, need %zu", workspace_bytes,
+                workspace, w.total);
+  if (w.total > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(PA_ERR_INVALID_ARG, "pa_append_decode: workspace must be 256-byte aligned");
+  pagedkv::DecodeParams p;
+  p.out = out;
+  p.q = q;
+  p.pool = kv_pool;
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.ws_acc = reinterpret_cast<float*>(workspace);
+  p.ws_ml = w.total ? reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + w.ml_offset) : nullptr;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.slot_mapping = slot_mapping;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_seqs = num_seqs;
+  p.num_heads = num_heads;
+  p.num_kv_heads = pool.num_kv_heads;
+  p.group = G;
+  p.num_blocks = pool.num_blocks;
+  p.max_seq_len = max_seq_len;
+  p.partition_tokens = partition_tokens_for(num_seqs, pool, max_seq_len > 0 ? max_seq_len : 1);
+  p.max_partitions = w.partitions > 0 ? w.partitions : 1;
+  p.scale_log2 = scale * pagedkv::kLog2e;
+  return pagedkv::launch_staged_bf16_d128(p, (cudaStream_t)stream);
 }
 
 pa_status pa_copy_blocks(void* kv_pool, const int32_t* src, const int32_t* dst, int32_t n,
