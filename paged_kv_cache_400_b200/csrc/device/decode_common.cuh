@@ -23,6 +23,8 @@ struct DecodeParams {
   const void* k_new;            // fused append: [B][Hkv][D] new token K (or null)
   const void* v_new;            // fused append: [B][Hkv][D] new token V
   const int64_t* slot_mapping;  // fused append: [B] slot of each new token
+  int32_t* work_items;          // persistent decode: (b << 16 | part) items, or null
+  int32_t* work_header;         // [0] item count, [1] next-item counter
   int32_t max_blocks;
   int32_t num_seqs;
   int32_t num_heads;

@@ -12,7 +12,12 @@
 // one 16-byte column fall in 8 different bank groups: ldmatrix and 16-byte
 // shared loads run without bank conflicts.
 //
-// CTA = (partition, KV head g, sequence b), 4 warps. Warp w owns the
+// Work unit = (partition, KV head g, sequence b), one CTA of 4 warps at a
+// time. Without split partitions the grid has one CTA per unit; with them, a
+// one-CTA plan kernel lists the non-empty units (full partitions first, then
+// the sequences' last partitions by decreasing size) and a grid of resident
+// CTAs takes units from that list through an atomic counter, so empty
+// partitions cost nothing and the smallest units finish last. Warp w owns the
 // partition's blocks w, w+4, w+8, ...; it runs its own ring of 2 stages with
 // one mbarrier each, issuing the TMA for its next block as soon as a stage is
 // consumed, so each warp keeps up to 16 KB in flight and a CTA 64 KB. Every
@@ -62,37 +67,32 @@ __device__ __forceinline__ uint32_t tile_chunk(int kv, int token, int chunk16) {
   return (uint32_t)((chunk16 >> 3) * 4096 + kv * 2048 + token * 128 + (((chunk16 & 7) ^ (token & 7)) << 4));
 }
 
-template <bool kMMA, bool kAppend>
-__global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constant__ CUtensorMap tmap,
-                                                            DecodeParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[kStagedWarps][kStagedStages];
-  __shared__ float red_m[kStagedWarps][16];
-  __shared__ float red_l[kStagedWarps][16];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+// Shared-memory state of a decode CTA (static part; the stages are dynamic).
+struct StagedShared {
+  uint64_t bars[kStagedWarps][kStagedStages];
+  float red_m[kStagedWarps][16];
+  float red_l[kStagedWarps][16];
+  int32_t next_item;
+};
 
-  const int32_t part = blockIdx.x;
-  const int32_t g = blockIdx.y;
-  const int32_t b = blockIdx.z;
+// Attention over partition `part` of sequence b for KV head g (all G query
+// heads). `phase` holds, per stage of this warp, the parity of its mbarrier's
+// next phase; it carries over between partitions of a persistent CTA.
+template <bool kMMA, bool kAppend>
+__device__ __forceinline__ void decode_partition(const CUtensorMap& tmap, const DecodeParams& p, uint8_t* smem,
+                                                 StagedShared& sh, int32_t part, int32_t g, int32_t b,
+                                                 int32_t L, uint32_t& phase) {
   const int32_t warp = threadIdx.x >> 5;
   const int32_t lane = threadIdx.x & 31;
   const int32_t G = p.group;
   const int32_t H = p.num_heads;
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
-  // the partition merge may be scheduled as soon as every CTA has started; it
-  // waits for this grid's completion before reading any partition state
-  grid_dependents_launch();
+  auto& bars = sh.bars;
+  auto& red_m = sh.red_m;
+  auto& red_l = sh.red_l;
 
-  const int32_t L = checked_len(p, b, part == 0 && g == 0 && threadIdx.x == 0);
   const int32_t S = p.partition_tokens;
   const int32_t nparts = (L + S - 1) / S;
-  if (L == 0) {
-    if (part == 0)
-      for (int32_t i = threadIdx.x; i < G * 128; i += blockDim.x)
-        out[((size_t)b * H + (size_t)g * G) * 128 + i] = __float2bfloat16_rn(0.f);
-    return;
-  }
-  if (part >= nparts) return;
   const int32_t t0 = part * S;
   const int32_t t1 = min(t0 + S, L);
   const int32_t nb = (t1 - t0 + 15) >> 4;
@@ -100,14 +100,6 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constan
   uint8_t* wsm = smem + warp * kStagedStages * kStageBytes;
   const uint32_t wsm_addr = smem_addr(wsm);
   const int32_t* table = p.block_tables + (size_t)b * p.max_blocks + (t0 >> 4);
-
-  if (lane == 0) {
-#pragma unroll
-    for (int s = 0; s < kStagedStages; ++s) mbar_init(&bars[warp][s], 1);
-    fence_barrier_init();
-    if (warp == 0) prefetch_tensormap(&tmap);
-  }
-  __syncwarp();
 
   // Block ids of this warp's blocks, read once: lane i holds the id of the
   // warp's i-th block (partition block warp + 4i), so issuing a load never
@@ -201,9 +193,10 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constan
 
   for (int32_t i = 0; i < my; ++i) {
     const int32_t s = i % kStagedStages;
-    if (!mbar_wait_bounded(&bars[warp][s], (uint32_t)(i / kStagedStages) & 1u, kWaitLimitNs)) {
+    if (!mbar_wait_bounded(&bars[warp][s], (phase >> s) & 1u, kWaitLimitNs)) {
       if (lane == 0) raise_device_error(PA_DEVERR_TIMEOUT);
     }
+    phase ^= 1u << s;
     const int32_t tok0 = t0 + (warp + i * kStagedWarps) * 16;
     const int32_t nvalid = min(16, t1 - tok0);
     const bool valid = (valid_mask >> s) & 1u;
@@ -421,6 +414,120 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constan
   }
 }
 
+// Grid mode (work_items == null): CTA = (partition, KV head, sequence).
+// Persistent mode: a grid of resident CTAs takes (sequence, partition, KV
+// head) items from the plan kernel's list, largest partitions first, through
+// an atomic counter, so no CTA is spent on an empty partition and the last
+// items to finish are the smallest.
+template <bool kMMA, bool kAppend>
+__global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constant__ CUtensorMap tmap,
+                                                            DecodeParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ StagedShared sh;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int32_t warp = threadIdx.x >> 5;
+  const int32_t lane = threadIdx.x & 31;
+  // the partition merge may be scheduled as soon as every CTA has started; it
+  // waits for this grid's completion before reading any partition state
+  grid_dependents_launch();
+  int32_t grid_len = 0;
+  if (p.work_items == nullptr) {
+    // grid mode: leave at once when this partition is empty (most CTAs of
+    // short sequences), before any set-up
+    const int32_t part = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    grid_len = checked_len(p, b, part == 0 && g == 0 && threadIdx.x == 0);
+    if (grid_len == 0) {
+      if (part == 0) {
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+        for (int32_t i = threadIdx.x; i < p.group * 128; i += blockDim.x)
+          out[((size_t)b * p.num_heads + (size_t)g * p.group) * 128 + i] = __float2bfloat16_rn(0.f);
+      }
+      return;
+    }
+    if (part >= (grid_len + p.partition_tokens - 1) / p.partition_tokens) return;
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < kStagedStages; ++s) mbar_init(&sh.bars[warp][s], 1);
+    fence_barrier_init();
+    if (warp == 0) prefetch_tensormap(&tmap);
+  }
+  __syncwarp();
+  uint32_t phase = 0;
+  if (p.work_items == nullptr) {
+    decode_partition<kMMA, kAppend>(tmap, p, smem, sh, blockIdx.x, blockIdx.y, blockIdx.z, grid_len, phase);
+    return;
+  }
+  grid_dependency_wait();  // the plan kernel's item list is complete
+  const int32_t total = __ldcg(p.work_header) * p.num_kv_heads;
+  if (threadIdx.x == 0) sh.next_item = atomicAdd(p.work_header + 1, 1);
+  __syncthreads();
+  int32_t item = sh.next_item;
+  while (item < total) {
+    int32_t next = 0;
+    if (threadIdx.x == 0) next = atomicAdd(p.work_header + 1, 1);  // in flight during the item
+    const int32_t bp = __ldcg(p.work_items + item / p.num_kv_heads);
+    const int32_t g = item % p.num_kv_heads;
+    const int32_t b = bp >> 16;
+    decode_partition<kMMA, kAppend>(tmap, p, smem, sh, bp & 0xffff, g, b, checked_len(p, b, false), phase);
+    // this item's shared-memory reads (generic proxy) precede the next item's
+    // TMA writes (async proxy)
+    fence_proxy_async_smem();
+    if (threadIdx.x == 0) sh.next_item = next;
+    __syncthreads();
+    item = sh.next_item;
+  }
+}
+
+// Work list for the persistent mode, one CTA: every non-empty partition of
+// every sequence as (b << 16 | part), full partitions first, then each
+// sequence's last partition by decreasing size (counting sort on the size in
+// blocks). Also raises PA_DEVERR_SEQLEN for bad lengths, writes zeros for
+// sequences of length 0, and resets the item counter.
+constexpr int kPlanThreads = 1024;
+
+__global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams p) {
+  __shared__ int32_t cnt[33];
+  __shared__ int32_t off[33];
+  // the decode CTAs may start (and set up) now; they wait for this grid's
+  // completion before reading the list
+  grid_dependents_launch();
+  const int32_t SB = p.partition_tokens >> 4;  // blocks per full partition (<= 32)
+  for (int32_t i = threadIdx.x; i <= SB; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  for (int32_t b = threadIdx.x; b < p.num_seqs; b += blockDim.x) {
+    const int32_t L = checked_len(p, b, true);
+    if (L == 0) {
+      uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)b * p.num_heads * 128);
+      for (int32_t i = 0; i < p.num_heads * 16; ++i) o[i] = make_uint4(0, 0, 0, 0);
+      continue;
+    }
+    const int32_t n = (L + p.partition_tokens - 1) / p.partition_tokens;
+    const int32_t r = ((L + 15) >> 4) - (n - 1) * SB;
+    if (n > 1) atomicAdd(&cnt[SB], n - 1);
+    atomicAdd(&cnt[r], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t acc = 0;
+    for (int32_t sz = SB; sz >= 1; --sz) {
+      off[sz] = acc;
+      acc += cnt[sz];
+    }
+    p.work_header[0] = acc;
+    p.work_header[1] = 0;
+  }
+  __syncthreads();
+  for (int32_t b = threadIdx.x; b < p.num_seqs; b += blockDim.x) {
+    const int32_t L = checked_len(p, b, false);
+    if (L == 0) continue;
+    const int32_t n = (L + p.partition_tokens - 1) / p.partition_tokens;
+    const int32_t r = ((L + 15) >> 4) - (n - 1) * SB;
+    for (int32_t part = 0; part + 1 < n; ++part) p.work_items[atomicAdd(&off[SB], 1)] = (b << 16) | part;
+    p.work_items[atomicAdd(&off[r], 1)] = (b << 16) | (n - 1);
+  }
+}
+
 // ---- host side ---------------------------------------------------------------
 
 inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -454,11 +561,42 @@ inline pa_status encode_pool_map(const DecodeParams& p, CUtensorMap* map) {
   return PA_OK;
 }
 
+// Launches one decode_staged_kernel variant: the grid-mode grid, or in
+// persistent mode min(items, resident CTAs) CTAs as a programmatic dependent
+// of the plan kernel.
 template <bool kMMA, bool kAppend>
-inline pa_status prepare_staged() {
-  static cudaError_t e = cudaFuncSetAttribute(decode_staged_kernel<kMMA, kAppend>,
-                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kStagedSmem);
-  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode: %s", cudaGetErrorString(e));
+inline pa_status launch_staged_variant(const CUtensorMap& map, const DecodeParams& p, cudaStream_t st) {
+  static int32_t per_sm = -1;
+  if (per_sm < 0) {
+    int32_t n = 0;
+    cudaError_t e = cudaFuncSetAttribute(decode_staged_kernel<kMMA, kAppend>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kStagedSmem);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_staged_kernel<kMMA, kAppend>, 128, kStagedSmem);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode: %s", cudaGetErrorString(e));
+    per_sm = n > 0 ? n : 1;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = kStagedSmem;
+  cfg.stream = st;
+  if (p.work_items == nullptr) {
+    cfg.gridDim = dim3(p.max_partitions, p.num_kv_heads, p.num_seqs);
+  } else {
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t most = (int64_t)p.num_seqs * p.max_partitions * p.num_kv_heads;
+    const int64_t resident = (int64_t)per_sm * (sms > 0 ? sms : 148);
+    cfg.gridDim = dim3((unsigned)(most < resident ? most : resident));
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_staged_kernel<kMMA, kAppend>, map, p);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode: launch failed: %s", cudaGetErrorString(e));
   return PA_OK;
 }
 
@@ -466,23 +604,18 @@ inline pa_status launch_staged_bf16_d128(const DecodeParams& p, cudaStream_t st)
   CUtensorMap map;
   pa_status s = encode_pool_map(p, &map);
   if (s != PA_OK) return s;
-  dim3 grid(p.max_partitions, p.num_kv_heads, p.num_seqs);
-  const bool append = p.k_new != nullptr;
-  if (p.group == 1 && !append) {
-    if ((s = prepare_staged<false, false>()) != PA_OK) return s;
-    decode_staged_kernel<false, false><<<grid, 128, kStagedSmem, st>>>(map, p);
-  } else if (p.group == 1) {
-    if ((s = prepare_staged<false, true>()) != PA_OK) return s;
-    decode_staged_kernel<false, true><<<grid, 128, kStagedSmem, st>>>(map, p);
-  } else if (!append) {
-    if ((s = prepare_staged<true, false>()) != PA_OK) return s;
-    decode_staged_kernel<true, false><<<grid, 128, kStagedSmem, st>>>(map, p);
-  } else {
-    if ((s = prepare_staged<true, true>()) != PA_OK) return s;
-    decode_staged_kernel<true, true><<<grid, 128, kStagedSmem, st>>>(map, p);
+  if (p.work_items != nullptr) {
+    decode_plan_kernel<<<1, kPlanThreads, 0, st>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode (plan): launch failed: %s", cudaGetErrorString(e));
   }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode: launch failed: %s", cudaGetErrorString(e));
+  const bool append = p.k_new != nullptr;
+  if (p.group == 1 && !append) s = launch_staged_variant<false, false>(map, p, st);
+  else if (p.group == 1) s = launch_staged_variant<false, true>(map, p, st);
+  else if (!append) s = launch_staged_variant<true, false>(map, p, st);
+  else s = launch_staged_variant<true, true>(map, p, st);
+  if (s != PA_OK) return s;
+  cudaError_t e = cudaSuccess;
   if (p.max_partitions <= 1) return PA_OK;
   e = launch_partition_merge<__nv_bfloat16, 128>(p, st);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode (merge): launch failed: %s", cudaGetErrorString(e));

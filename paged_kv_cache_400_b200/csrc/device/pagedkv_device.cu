@@ -17,6 +17,11 @@ using pagedkv::fail;
 namespace {
 
 constexpr int32_t kNumSMs = 148;
+// From this many partitions per sequence (a long max_seq_len) the staged
+// decode runs as a persistent grid over a work list instead of one CTA per
+// (partition, head, sequence): most CTAs of short sequences would be empty.
+// Below it the plain grid is faster (no plan launch, no per-item latency).
+constexpr int32_t kWorkListPartitions = 32;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -51,20 +56,24 @@ int32_t partition_tokens_for(int32_t num_seqs, const pa_pool_desc& pool, int32_t
 }
 
 struct WorkspaceLayout {
-  size_t acc_bytes, ml_offset, total;
+  size_t acc_bytes, ml_offset, items_offset, header_offset, total;
   int32_t partitions;
 };
 
 WorkspaceLayout workspace_layout(int32_t num_seqs, int32_t num_heads, const pa_pool_desc& pool,
                                  int32_t max_seq_len) {
-  WorkspaceLayout w{0, 0, 0, 0};
+  WorkspaceLayout w{0, 0, 0, 0, 0, 0};
   const int32_t S = partition_tokens_for(num_seqs, pool, max_seq_len);
   w.partitions = (max_seq_len + S - 1) / S;
   if (w.partitions <= 1) return w;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   const size_t units = (size_t)num_seqs * num_heads * w.partitions;
   w.acc_bytes = units * pool.head_dim * sizeof(float);
-  w.ml_offset = (w.acc_bytes + 255) & ~(size_t)255;
-  w.total = w.ml_offset + units * 2 * sizeof(float);
+  w.ml_offset = up(w.acc_bytes);
+  // work list of the persistent decode: one int per (sequence, partition)
+  w.items_offset = up(w.ml_offset + units * 2 * sizeof(float));
+  w.header_offset = up(w.items_offset + (size_t)num_seqs * w.partitions * sizeof(int32_t));
+  w.total = w.header_offset + 2 * sizeof(int32_t);
   return w;
 }
 
@@ -184,6 +193,10 @@ pa_status pa_decode(void* out, const void* q, const void* kv_pool, const int32_t
   p.k_new = nullptr;
   p.v_new = nullptr;
   p.slot_mapping = nullptr;
+  const bool use_list = w.total && w.partitions >= kWorkListPartitions;
+  p.work_items = use_list ? reinterpret_cast<int32_t*>(reinterpret_cast<char*>(workspace) + w.items_offset) : nullptr;
+  p.work_header =
+      use_list ? reinterpret_cast<int32_t*>(reinterpret_cast<char*>(workspace) + w.header_offset) : nullptr;
   p.max_blocks = max_blocks_per_seq;
   p.num_seqs = num_seqs;
   p.num_heads = num_heads;
@@ -262,6 +275,10 @@ pa_status pa_append_decode(void* out, const void* q, const void* k_new, const vo
   p.k_new = k_new;
   p.v_new = v_new;
   p.slot_mapping = slot_mapping;
+  const bool use_list = w.total && w.partitions >= kWorkListPartitions;
+  p.work_items = use_list ? reinterpret_cast<int32_t*>(reinterpret_cast<char*>(workspace) + w.items_offset) : nullptr;
+  p.work_header =
+      use_list ? reinterpret_cast<int32_t*>(reinterpret_cast<char*>(workspace) + w.header_offset) : nullptr;
   p.max_blocks = max_blocks_per_seq;
   p.num_seqs = num_seqs;
   p.num_heads = num_heads;

@@ -133,6 +133,20 @@ def test_long_sequences_many_partitions():
     check_case(case)
 
 
+@pytest.mark.parametrize("max_seq_len", [16384, 65536])
+def test_long_max_context_uses_the_work_list(max_seq_len):
+    # >= 32 partitions per sequence: persistent decode over the plan kernel's list
+    lens = [1, 17, 512, 513, 3000, 9000, 16384, 5, 0, 700] if max_seq_len == 16384 else \
+        [70000 // 2, 33, 1, 1025, 40000]
+    lens = [n for n in lens if n >= 1]
+    width = max_seq_len // 16
+    case = wl.custom_case(f"wl_{max_seq_len}", 17, lens, 8192, 32, 8, 128, "bf16", width, max_seq_len)
+    check_case(case)
+    mha = wl.custom_case(f"wl_mha_{max_seq_len}", 18, [3, 4000, 12000], 2048, 32, 32, 128, "bf16", width,
+                         max_seq_len)
+    check_case(mha)
+
+
 def test_single_token_sequences():
     case = wl.custom_case("ones", 12, [1] * 40, 128, 32, 8, 128, "bf16", 4, 64)
     _, _, out, _ = check_case(case)
