@@ -456,6 +456,14 @@ def run_ours(args, rank, world, dist):
             "sample": f"{done} of {B} sequences (random order), one decode token each: oracle "
                       f"copy-on-write + append + gather through its own block tables + fp64 "
                       f"attention, {el:.1f} s of oracle time"}
+        try:
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(1):
+                d1, e1 = oracle_sample(case, args.cpu_seconds / 3, rng_seed=1)
+            line["cpu_baseline"]["one_core_value"] = d1 / e1
+        except Exception as e:  # pragma: no cover
+            line["cpu_baseline"]["one_core_value"] = None
+            line["cpu_baseline"]["one_core_error"] = repr(e)
     print(json.dumps(line), flush=True)
 
 

@@ -485,14 +485,15 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constan
 // blocks). Also raises PA_DEVERR_SEQLEN for bad lengths, writes zeros for
 // sequences of length 0, and resets the item counter.
 constexpr int kPlanThreads = 1024;
+constexpr int kMaxPartitionBlocks = 128;  // partitions of at most 2048 tokens
 
 __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams p) {
-  __shared__ int32_t cnt[33];
-  __shared__ int32_t off[33];
+  __shared__ int32_t cnt[kMaxPartitionBlocks + 1];
+  __shared__ int32_t off[kMaxPartitionBlocks + 1];
   // the decode CTAs may start (and set up) now; they wait for this grid's
   // completion before reading the list
   grid_dependents_launch();
-  const int32_t SB = p.partition_tokens >> 4;  // blocks per full partition (<= 32)
+  const int32_t SB = p.partition_tokens >> 4;  // blocks per full partition (<= kMaxPartitionBlocks)
   for (int32_t i = threadIdx.x; i <= SB; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
   for (int32_t b = threadIdx.x; b < p.num_seqs; b += blockDim.x) {

@@ -17,11 +17,15 @@ using pagedkv::fail;
 namespace {
 
 constexpr int32_t kNumSMs = 148;
-// From this many partitions per sequence (a long max_seq_len) the staged
-// decode runs as a persistent grid over a work list instead of one CTA per
-// (partition, head, sequence): most CTAs of short sequences would be empty.
-// Below it the plain grid is faster (no plan launch, no per-item latency).
-constexpr int32_t kWorkListPartitions = 32;
+// From this many partitions per sequence the staged decode runs as a
+// persistent grid over a work list (largest partitions first) instead of one
+// CTA per (partition, head, sequence): most grid CTAs of short sequences would
+// be empty, and a few long sequences would finish last. Below it the plain
+// grid is faster (no plan launch, no per-item latency).
+#ifndef PA_WORKLIST_PARTITIONS
+#define PA_WORKLIST_PARTITIONS 4
+#endif
+constexpr int32_t kWorkListPartitions = PA_WORKLIST_PARTITIONS;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -46,10 +50,17 @@ pa_status launch_status(const char* fn) {
   return PA_OK;
 }
 
+#ifndef PA_PARTITION_TOKENS
+#define PA_PARTITION_TOKENS 2048
+#endif
+static_assert(PA_PARTITION_TOKENS % 16 == 0 && PA_PARTITION_TOKENS / 16 <= pagedkv::kMaxPartitionBlocks,
+              "partition of whole blocks, at most 2048 tokens (a warp holds at most 32 block ids)");
+
 int32_t partition_tokens_for(int32_t num_seqs, const pa_pool_desc& pool, int32_t max_seq_len) {
-  // 512-token partitions; halve while the grid would not give every SM a few
-  // CTAs, down to 128.
-  int32_t S = 512;
+  // PA_PARTITION_TOKENS-token partitions (2048 unless built otherwise: large
+  // partitions keep the partial states and their merge small); halve while
+  // the grid would not give every SM a few CTAs, down to 128.
+  int32_t S = PA_PARTITION_TOKENS;
   const int64_t pairs = (int64_t)num_seqs * pool.num_kv_heads;
   while (S > 128 && pairs * ((max_seq_len + S - 1) / S) < 4 * kNumSMs) S /= 2;
   return S;

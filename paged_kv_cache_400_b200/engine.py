@@ -4,7 +4,8 @@ Each step the host scheduler (pa_sched_step, C++) decides which requests run,
 which are admitted (their prompt K/V are (re)written: recompute), which grow a
 block, which are preempted or finish; then, for every layer, the step's device
 work runs through the C ABI: copy-on-write block copies, the prompt-token
-append, the decode-token append, and paged decode over the running batch
+append, then the decode-token append and paged decode over the running batch
+in one call (pa_append_decode)
 ("vLLM 原理：PagedAttention 和 Continuous Batching" / "vLLM 的调度 / 调度流程";
 "大模型推理性能优化：PagedAttention与Continuous Batching原理与实践" §2.3).
 
@@ -69,7 +70,7 @@ class DecodeEngine:
         shape = (num_blocks, 2, num_kv_heads, bd.BLOCK_SIZE, head_dim)
         self.pools = [torch.empty(shape, dtype=dtype, device=self.device) for _ in range(num_layers)]
         self._ws = None
-        self._ws_batch = 0
+        self._ws_bytes = 0
 
     def close(self):
         self.sched.close()
@@ -117,9 +118,14 @@ class DecodeEngine:
 
     # ---- device side -------------------------------------------------------------
     def workspace(self, batch):
-        if self._ws is None or batch > self._ws_batch:
-            self._ws = bd.alloc_workspace(batch, self.num_heads, self.pools[0], self.max_seq_len)
-            self._ws_batch = batch
+        """A workspace large enough for `batch` sequences (grown on demand: the
+        partition size, hence the bytes needed, depends on the batch)."""
+        need = bd.pa_decode_workspace_size(batch, self.num_heads, self.pools[0], self.max_seq_len)
+        if need == 0:
+            return None
+        if self._ws is None or need > self._ws_bytes:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+            self._ws_bytes = need
         return self._ws
 
     def run_layers(self, idx: StepIndices, inputs, out=None):
@@ -149,6 +155,7 @@ class DecodeEngine:
                 bd.pa_copy_blocks(pool, cs, cd)
             if ps is not None:
                 bd.pa_reshape_and_cache(x["k_prompt"], x["v_prompt"], pool, ps)
-            bd.pa_reshape_and_cache(x["k_dec"], x["v_dec"], pool, ds)
-            bd.pa_decode(outs[l], x["q"], pool, bt, sl, self.scale, self.max_seq_len, ws)
+            # each running request's new token appended and attended in one call
+            bd.pa_append_decode(outs[l], x["q"], x["k_dec"], x["v_dec"], pool, ds, bt, sl, self.scale,
+                                self.max_seq_len, ws)
         return outs

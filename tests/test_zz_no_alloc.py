@@ -54,11 +54,12 @@ def test_noalloc_matches_workspace_decode_twice(heads, kv_heads):
 def test_noalloc_rejects_shapes_beyond_its_array():
     case = wl.custom_case("noalloc_big", 22, [16] * 4, 64, 32, 8, 128, "bf16", 4, 64)
     pool, q, bt, sl = _inputs(case)
-    q_big = torch.empty(256, 32, 128, dtype=torch.bfloat16, device=DEV)
-    need = pk.pa_decode_workspace_size(256, 32, pool, 8192)
+    B, max_len = 1024, 32768   # 1024 sequences of up to 32k tokens: partials beyond 32 MiB
+    q_big = torch.empty(B, 32, 128, dtype=torch.bfloat16, device=DEV)
+    need = pk.pa_decode_workspace_size(B, 32, pool, max_len)
     assert need > (32 << 20)
     with pytest.raises(bd.PagedKVError) as e:
         bd.pa_decode_noalloc(q_big.clone(), q_big, pool,
-                             torch.zeros(256, 512, dtype=torch.int32, device=DEV),
-                             torch.zeros(256, dtype=torch.int32, device=DEV), 0.1, 8192)
+                             torch.zeros(B, max_len // 16, dtype=torch.int32, device=DEV),
+                             torch.zeros(B, dtype=torch.int32, device=DEV), 0.1, max_len)
     assert e.value.status == "WORKSPACE"
