@@ -51,6 +51,8 @@ def parse_args():
                     help="gqa is the benchmark line; the others are extra measurements")
     ap.add_argument("--trace-layers", type=int, default=32)
     ap.add_argument("--trace-requests", type=int, default=2000)
+    ap.add_argument("--graphs", action="store_true",
+                    help="trace: replay each step's decode over all layers as a CUDA graph")
     ap.add_argument("--batch", type=int, default=256,
                     help="sequences per GPU (256 is the workload; smaller only for profiling captures)")
     ap.add_argument("--e2e-steps", type=int, default=None)
@@ -487,6 +489,10 @@ def run_trace(args, rank, world):
     tr = wl.trace_case(args.seed + rank, n_requests=args.trace_requests, num_layers=args.trace_layers)
     eng = DecodeEngine(tr.num_blocks, tr.num_layers, tr.num_heads, tr.num_kv_heads, tr.head_dim,
                        tr.arrival_step, tr.prompt_len, tr.output_len, tr.table_width, tr.scale, dev)
+    graphed = None
+    if args.graphs:
+        from paged_kv_cache_400_b200.engine import GraphedLayers
+        graphed = GraphedLayers(eng, max_batch=1280)
     stream = torch.cuda.current_stream()
     events = []
     tokens = kv_tokens = prompt_tokens = steps = preempted = 0
@@ -502,12 +508,18 @@ def run_trace(args, rank, world):
         n = len(idx.running)
         if n:
             reqs_p, pos_p = eng.prompt_positions(idx)
-            inputs = tr.step_inputs(idx.step, idx.running, idx.seq_lens, reqs_p, pos_p, dev)
+            inputs, stacked = tr.step_inputs(idx.step, idx.running, idx.seq_lens, reqs_p, pos_p, dev,
+                                             stacked=True)
+            if graphed is not None:
+                graphed._graph(((n + graphed.bucket - 1) // graphed.bucket) * graphed.bucket)
             torch.cuda.synchronize()
             t2 = time.perf_counter()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            eng.run_layers(idx, inputs)
+            if graphed is not None:
+                graphed.run(idx, inputs, stacked)
+            else:
+                eng.run_layers(idx, inputs)
             e1.record(stream)
             torch.cuda.synchronize()
             e2e_s += (t1 - t0) + (time.perf_counter() - t2)
@@ -526,6 +538,7 @@ def run_trace(args, rank, world):
     eng.close()
     kv_bytes = kv_tokens * 2 * tr.num_kv_heads * tr.head_dim * 2 * tr.num_layers
     line = {
+        "graphs": bool(args.graphs),
         "workload": f"continuous-batching trace: {args.trace_requests} requests, Poisson(50) arrivals/step, "
                     "prompts U[16,1024], outputs geometric mean 200 cap 2048, 40000-block pools, "
                     f"{tr.num_layers} layers x (prompt append + decode-token append + paged decode), "

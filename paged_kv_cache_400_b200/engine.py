@@ -159,3 +159,100 @@ class DecodeEngine:
             bd.pa_append_decode(outs[l], x["q"], x["k_dec"], x["v_dec"], pool, ds, bt, sl, self.scale,
                                 self.max_seq_len, ws)
         return outs
+
+
+class GraphedLayers:
+    """The decode part of a step over all layers (each running request's new
+    token appended and attended: pa_append_decode per layer) replayed as one
+    CUDA graph per batch-size bucket.
+
+    Padded rows have length 0 and slot -1: they append nothing and their
+    output rows are zeros, so a bucket's graph serves any batch up to its size.
+    Index arrays and per-layer inputs are copied into the graph's static
+    buffers before each replay; prompt appends and copy-on-write copies (their
+    sizes vary every step) run eagerly before it. Capture happens on first use
+    of a bucket, after an eager warm-up of the same calls.
+    """
+
+    def __init__(self, engine: "DecodeEngine", max_batch: int, bucket: int = 64):
+        self.eng = engine
+        self.bucket = bucket
+        self.max_batch = ((max_batch + bucket - 1) // bucket) * bucket
+        dev, L = engine.device, engine.num_layers
+        H, Hkv, D, W = engine.num_heads, engine.num_kv_heads, engine.head_dim, engine.table_width
+        dt = engine.pools[0].dtype
+        B = self.max_batch
+        self.q = torch.zeros(L, B, H, D, dtype=dt, device=dev)
+        self.k = torch.zeros(L, B, Hkv, D, dtype=dt, device=dev)
+        self.v = torch.zeros(L, B, Hkv, D, dtype=dt, device=dev)
+        self.out = torch.zeros(L, B, H, D, dtype=dt, device=dev)
+        self.bt = torch.full((B, W), -1, dtype=torch.int32, device=dev)
+        self.sl = torch.zeros(B, dtype=torch.int32, device=dev)
+        self.slots = torch.full((B,), -1, dtype=torch.int64, device=dev)
+        need = max(bd.pa_decode_workspace_size(n, H, engine.pools[0], engine.max_seq_len)
+                   for n in range(bucket, B + 1, bucket))
+        self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        self.graphs = {}
+
+    def _calls(self, n):
+        e = self.eng
+        for l, pool in enumerate(e.pools):
+            bd.pa_append_decode(self.out[l, :n], self.q[l, :n], self.k[l, :n], self.v[l, :n], pool,
+                                self.slots[:n], self.bt[:n], self.sl[:n], e.scale, e.max_seq_len, self.ws)
+
+    def _graph(self, n):
+        g = self.graphs.get(n)
+        if g is None:
+            # eager warm-up (kernel attributes are set outside capture) on inert
+            # rows only: length 0 and slot -1 append and read nothing
+            self.sl[:n].zero_()
+            self.slots[:n].fill_(-1)
+            self._calls(n)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._calls(n)
+            self.graphs[n] = g
+        return g
+
+    def run(self, idx: StepIndices, inputs, stacked=None):
+        """inputs as for DecodeEngine.run_layers; `stacked` = (q [L][n][H][D],
+        k [L][n][Hkv][D], v [L][n][Hkv][D]) of the decode tokens, when the
+        caller has them in one tensor each (one copy each instead of per layer)."""
+        e = self.eng
+        dev = e.device
+        n = len(idx.running)
+        if n == 0:
+            return []
+        if n > self.max_batch:
+            raise ValueError(f"batch {n} above the graphed maximum {self.max_batch}")
+        nb = ((n + self.bucket - 1) // self.bucket) * self.bucket
+        graph = self._graph(nb)  # captured on first use, before the rows are filled
+        # eager, variable-size work first
+        cs = torch.from_numpy(idx.cow_src).to(dev) if len(idx.cow_src) else None
+        cd = torch.from_numpy(idx.cow_dst).to(dev) if len(idx.cow_dst) else None
+        ps = torch.from_numpy(idx.prompt_slots).to(dev, non_blocking=True) if len(idx.prompt_slots) else None
+        for l, pool in enumerate(e.pools):
+            if cs is not None:
+                bd.pa_copy_blocks(pool, cs, cd)
+            if ps is not None:
+                bd.pa_reshape_and_cache(inputs[l]["k_prompt"], inputs[l]["v_prompt"], pool, ps)
+        # static buffers: this step's rows, then inert padding up to the bucket
+        self.bt[:n].copy_(torch.from_numpy(idx.block_tables), non_blocking=True)
+        self.sl[:n].copy_(torch.from_numpy(idx.seq_lens), non_blocking=True)
+        self.slots[:n].copy_(torch.from_numpy(idx.decode_slots), non_blocking=True)
+        if nb > n:
+            self.bt[n:nb].fill_(-1)
+            self.sl[n:nb].zero_()
+            self.slots[n:nb].fill_(-1)
+        if stacked is not None:
+            self.q[:, :n].copy_(stacked[0])
+            self.k[:, :n].copy_(stacked[1])
+            self.v[:, :n].copy_(stacked[2])
+        else:
+            for l in range(e.num_layers):
+                self.q[l, :n].copy_(inputs[l]["q"])
+                self.k[l, :n].copy_(inputs[l]["k_dec"])
+                self.v[l, :n].copy_(inputs[l]["v_dec"])
+        graph.replay()
+        return [self.out[l, :n] for l in range(e.num_layers)]

@@ -307,7 +307,7 @@ class TraceCase:
         return x[:, 0].contiguous(), x[:, 1].contiguous()
 
     def step_inputs(self, step: int, running, seq_lens, prompt_reqs, prompt_pos, device,
-                    chunk_elems: int = 1 << 26):
+                    chunk_elems: int = 1 << 26, stacked: bool = False):
         """Per-layer inputs of one continuous-batching step: the query and the
         new token's K/V of each running request (position seq_len - 1), and the
         prompt K/V of the (re)admitted requests, generated layer by layer in
@@ -347,6 +347,8 @@ class TraceCase:
                 k_p = torch.cat([a for a, _ in parts])
                 v_p = torch.cat([b for _, b in parts])
             out.append({"q": q, "k_dec": k_d, "v_dec": v_d, "k_prompt": k_p, "v_prompt": v_p})
+        if stacked:
+            return out, (q_all, kv_all[:, :, 0], kv_all[:, :, 1])
         return out
 
     def q_values(self, layer: int, step: int, reqs, device="cpu"):

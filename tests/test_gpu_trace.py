@@ -90,3 +90,43 @@ def test_trace_with_preemption_matches_oracle():
     assert pk.pa_get_device_error() == 0
     assert preempted_seen > 0 and checked >= 20, (preempted_seen, checked, steps)
     eng.close()
+
+
+def test_graphed_layer_loop_matches_oracle():
+    """The same trace with each step's decode over all layers replayed as a CUDA
+    graph per batch bucket (padded rows inert)."""
+    from paged_kv_cache_400_b200.engine import GraphedLayers
+    trace = wl.trace_case(seed=6, n_requests=120, rate=12.0, num_blocks=1200, num_layers=2,
+                          output_cap=120)
+    eng = DecodeEngine(trace.num_blocks, trace.num_layers, trace.num_heads, trace.num_kv_heads,
+                       trace.head_dim, trace.arrival_step, trace.prompt_len, trace.output_len,
+                       trace.table_width, trace.scale, DEV)
+    graphed = GraphedLayers(eng, max_batch=128, bucket=32)
+    obm = OracleBlockManager(trace.num_blocks)
+    osch = OracleScheduler(obm, trace.arrival_step, trace.prompt_len, trace.output_len, trace.table_width)
+    rng = np.random.default_rng(1)
+    checked = 0
+    while True:
+        idx = eng.schedule()
+        o = osch.step()
+        if len(idx.running):
+            reqs_p, pos_p = eng.prompt_positions(idx)
+            inputs, stacked = trace.step_inputs(idx.step, idx.running, idx.seq_lens, reqs_p, pos_p, DEV,
+                                                stacked=True)
+            outs = graphed.run(idx, inputs, stacked)
+            if idx.step % 15 == 0 and checked < 30:
+                layer = int(rng.integers(0, trace.num_layers))
+                got = outs[layer].float().cpu().numpy()
+                for i in rng.choice(len(idx.running), size=min(3, len(idx.running)), replace=False):
+                    r = int(idx.running[i])
+                    ref = oracle_attention(trace, layer, idx.step, r,
+                                           o["block_tables"][i][:(o["seq_lens"][i] + 15) // 16],
+                                           o["seq_lens"][i])
+                    assert float(np.abs(got[i] - ref).max()) <= 1e-2
+                    checked += 1
+        if idx.done:
+            break
+    import paged_kv_cache_400_b200 as pk
+    assert pk.pa_get_device_error() == 0
+    assert checked >= 10 and len(graphed.graphs) >= 2
+    eng.close()
