@@ -47,10 +47,12 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--workload", choices=["gqa", "mha", "prefix", "trace"], default="gqa",
+    ap.add_argument("--workload", choices=["gqa", "mha", "prefix", "trace", "prefix_trace"], default="gqa",
                     help="gqa is the benchmark line; the others are extra measurements")
     ap.add_argument("--trace-layers", type=int, default=32)
     ap.add_argument("--trace-requests", type=int, default=2000)
+    ap.add_argument("--no-prefix-cache", action="store_true",
+                    help="prefix_trace: run without automatic prefix caching (for comparison)")
     ap.add_argument("--graphs", action="store_true",
                     help="trace: replay each step's decode over all layers as a CUDA graph")
     ap.add_argument("--batch", type=int, default=256,
@@ -486,16 +488,23 @@ def run_trace(args, rank, world):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    tr = wl.trace_case(args.seed + rank, n_requests=args.trace_requests, num_layers=args.trace_layers)
+    shared = args.workload == "prefix_trace"
+    if shared:
+        tr = wl.prefix_trace_case(args.seed + rank, n_requests=args.trace_requests,
+                                  num_layers=args.trace_layers)
+    else:
+        tr = wl.trace_case(args.seed + rank, n_requests=args.trace_requests, num_layers=args.trace_layers)
+    caching = shared and not args.no_prefix_cache
     eng = DecodeEngine(tr.num_blocks, tr.num_layers, tr.num_heads, tr.num_kv_heads, tr.head_dim,
-                       tr.arrival_step, tr.prompt_len, tr.output_len, tr.table_width, tr.scale, dev)
+                       tr.arrival_step, tr.prompt_len, tr.output_len, tr.table_width, tr.scale, dev,
+                       prompt_tokens=tr.prompt_tokens if caching else None)
     graphed = None
     if args.graphs:
         from paged_kv_cache_400_b200.engine import GraphedLayers
         graphed = GraphedLayers(eng, max_batch=1280)
     stream = torch.cuda.current_stream()
     events = []
-    tokens = kv_tokens = prompt_tokens = steps = preempted = 0
+    tokens = kv_tokens = prompt_tokens = steps = preempted = cached_tokens = peak_batch = 0
     host_s = e2e_s = 0.0
     sampler = ClockSampler(local)
     sampler.start()
@@ -529,6 +538,8 @@ def run_trace(args, rank, world):
             prompt_tokens += len(idx.prompt_slots)
         steps += 1
         preempted += idx.record.preempted
+        cached_tokens += int(idx.prompt_starts.sum())
+        peak_batch = max(peak_batch, n)
         if idx.done:
             break
     wall1 = time.perf_counter()
@@ -537,16 +548,22 @@ def run_trace(args, rank, world):
     gpu_s = sum(a.elapsed_time(b) for a, b in events) / 1e3
     eng.close()
     kv_bytes = kv_tokens * 2 * tr.num_kv_heads * tr.head_dim * 2 * tr.num_layers
+    prompts = ("8 shared system prompts U[256,1024] + user tokens U[16,512]" if shared
+               else "prompts U[16,1024]")
     line = {
         "graphs": bool(args.graphs),
+        "prefix_caching": caching,
         "workload": f"continuous-batching trace: {args.trace_requests} requests, Poisson(50) arrivals/step, "
-                    "prompts U[16,1024], outputs geometric mean 200 cap 2048, 40000-block pools, "
+                    f"{prompts}, outputs geometric mean 200 cap 2048, 40000-block pools, "
                     f"{tr.num_layers} layers x (prompt append + decode-token append + paged decode), "
                     "32/8 heads, head_dim 128, bf16",
+        "prompt_tokens_cached": cached_tokens, "peak_batch": peak_batch,
         "metric": "generated tokens/s (device time of the layer loops)", "value": tokens / gpu_s,
         "unit": "tokens/s", "steps": steps, "generated_tokens": tokens, "prompt_tokens_written": prompt_tokens,
         "preemptions": preempted, "gpu_s": gpu_s, "host_scheduler_s": host_s,
         "kv_read_tb": kv_bytes / 1e12, "kv_read_gbs": kv_bytes / gpu_s / 1e9,
+        "kv_read_note": ("logical bytes: blocks shared by many sequences are read through L2"
+                         if caching else "every sequence's own blocks"),
         "e2e": {"value": tokens / e2e_s, "unit": "tokens/s",
                 "note": "pa_sched_step + index H2D + layer loops, wall clock; input generation excluded"},
         "wall_s": wall1 - wall0, "clocks": sampler.summary(wall0, wall1),
@@ -572,7 +589,7 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
-        elif args.workload == "trace":
+        elif args.workload in ("trace", "prefix_trace"):
             run_trace(args, rank, world)
         else:
             run_ours(args, rank, world, dist)

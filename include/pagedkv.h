@@ -316,6 +316,42 @@ pa_status pa_bm_pack(const pa_bm* bm, const int64_t* seqs, int32_t n,
                      int32_t max_blocks, int32_t* block_tables,
                      int32_t* seq_lens, int64_t* last_slots);
 
+/*
+ * Automatic prefix caching ([A] §3.4 "--enable-prefix-caching": requests with
+ * a common prompt prefix, e.g. the same system prompt, skip recomputing it;
+ * [B] "优势 / 3. 支持共享"). Off by default; switch it on for a fresh block
+ * manager. A full block of a prompt is identified by the chained hash
+ *     h_i = H(h_{i-1}, tokens[16i .. 16i+15]),   h_{-1} = 0,
+ * H(p, t) = x after x = mix(p ^ 0x9E3779B97F4A7C15) and x = mix(x ^ t_j) for
+ * each of the 16 token ids t_j (as uint32), mix being SplitMix64's output
+ * function. Cached blocks whose refcount drops to 0 stay reusable on an
+ * evictable list (least recently released first); a fresh block comes from
+ * the free list, else by evicting that list's head. A block's cache entry
+ * becomes reusable by others only once pa_bm_mark_written says its KV was
+ * written; a request freed before that leaves nothing cached.
+ */
+pa_status pa_bm_set_prefix_caching(pa_bm* bm, int32_t enable);
+/*
+ * pa_bm_allocate for a request whose first num_prompt_tokens tokens are
+ * prompt_tokens (num_tokens >= num_prompt_tokens tokens of KV in total): the
+ * longest run of leading full prompt blocks found in the cache is shared
+ * (refcount +1), the rest are fresh blocks; new full prompt blocks enter the
+ * cache. *cached_tokens = 16 x the leading shared blocks whose KV is already
+ * written (the caller writes KV from that position on). All or nothing
+ * (PA_ERR_NO_BLOCKS when the fresh blocks do not fit). Without prefix caching
+ * it is pa_bm_allocate with *cached_tokens = 0.
+ */
+pa_status pa_bm_allocate_prefix(pa_bm* bm, int64_t seq, const int32_t* prompt_tokens,
+                                int32_t num_prompt_tokens, int32_t num_tokens,
+                                int32_t* cached_tokens);
+/* The KV of seq's cached blocks has been written (enqueued): they may be reused. */
+pa_status pa_bm_mark_written(pa_bm* bm, int64_t seq);
+/* Cached blocks with refcount 0, next to evict first. pa_bm_num_free counts
+ * them as free. */
+pa_status pa_bm_evictable_list(const pa_bm* bm, int32_t* out, int32_t cap, int32_t* n);
+/* Number of blocks currently findable in the prefix cache. */
+int32_t pa_bm_num_cached(const pa_bm* bm);
+
 /* ------------------------------------------------------------------------ */
 /* Continuous-batching step loop ([A] §2.3, [B] "vLLM 的调度", "Preemption")  */
 /* ------------------------------------------------------------------------ */
@@ -339,8 +375,8 @@ typedef struct {
   int32_t num_prompt_tokens;
   const int64_t* prompt_seqs;   /* [num_prompt_seqs] request ids               */
   const int32_t* prompt_lens;   /* [num_prompt_seqs] tokens of KV (re)written  */
-  const int64_t* prompt_slots;  /* [num_prompt_tokens] positions 0..len-1 of
-                                   each prompt seq, in prompt_seqs order        */
+  const int64_t* prompt_slots;  /* [num_prompt_tokens] positions start..len-1
+                                   of each prompt seq, in prompt_seqs order     */
   int32_t num_cow;
   const int32_t* cow_src;       /* [num_cow] copy-on-write pairs, in order     */
   const int32_t* cow_dst;
@@ -352,6 +388,11 @@ typedef struct {
   const int64_t* finished;      /* retired at the start of this step           */
   int32_t num_waiting;          /* queue length after the step                 */
   int32_t num_free_blocks;      /* free blocks after the step                  */
+  const int32_t* prompt_starts; /* [num_prompt_seqs] first position written:
+                                   positions before it are in reused cached
+                                   blocks (0 without prefix caching); the
+                                   request's prompt_slots cover [start, len)  */
+  int32_t num_cached_tokens;    /* sum of prompt_starts this step              */
 } pa_step_out;
 
 /*
@@ -387,6 +428,15 @@ pa_status pa_sched_create(pa_bm* bm, const int32_t* arrival_step,
  * with out->done = 1 and nothing running. PA_ERR_NO_BLOCKS if the waiting head
  * cannot fit even with nothing running (the pool is too small for it). */
 pa_status pa_sched_step(pa_sched* s, pa_step_out* out);
+/*
+ * Gives the scheduler the prompt token ids (request i's prompt is
+ * tokens[offsets[i] .. offsets[i] + prompt_len[i])), switching admission to
+ * pa_bm_allocate_prefix: a (re)admitted request reuses the cached blocks of
+ * its prompt's longest cached prefix and only the KV after it is written
+ * (prompt_starts). Requires the block manager's prefix caching; call before
+ * the first step. Arrays are copied.
+ */
+pa_status pa_sched_set_prompt_tokens(pa_sched* s, const int32_t* tokens, const int64_t* offsets);
 void pa_sched_destroy(pa_sched* s);
 
 #ifdef __cplusplus

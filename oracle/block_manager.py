@@ -19,6 +19,15 @@ Sources:
       page list; new requests take pages from it; different logical blocks may
       map to one physical page.
 
+Prefix caching ("PagedAttention与Continuous Batching原理与实践" §3.4: with
+--enable-prefix-caching, requests sharing a prompt prefix such as a system
+prompt avoid recomputing it) is read as: full prompt blocks are keyed by the
+chained hash of (previous blocks' hash, their 16 token ids); allocation shares
+the longest run of cached leading blocks; a cached block whose refcount drops
+to 0 stays findable on an evictable list (least recently released first) and
+a fresh block comes from the free list, else by evicting that list's head; a
+cached block may be reused only after its KV was written (mark_written).
+
 Readings where the pages are silent (each also listed in the design notes):
   * allocation is all-or-nothing (the deque code would fail half way);
   * freed blocks go to the free-list tail in table order;
@@ -30,9 +39,10 @@ Readings where the pages are silent (each also listed in the design notes):
 """
 from __future__ import annotations
 
-from collections import deque
+from collections import OrderedDict, deque
 
 BLOCK_SIZE = 16
+_M64 = (1 << 64) - 1
 
 
 class BMError(Exception):
@@ -42,6 +52,23 @@ class BMError(Exception):
     def __init__(self, status: str, msg: str = ""):
         super().__init__(f"{status}: {msg}")
         self.status = status
+
+
+def mix64(z: int) -> int:
+    """SplitMix64's output function (Stafford's "Mix13" 64-bit finaliser)."""
+    z &= _M64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _M64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _M64
+    return z ^ (z >> 31)
+
+
+def chain_hash(parent: int, tokens) -> int:
+    """Hash of a full block of 16 token ids given the hash of the prompt before
+    it (0 for the first block): one mix of the parent, then one per token."""
+    x = mix64(parent ^ 0x9E3779B97F4A7C15)
+    for t in tokens:
+        x = mix64(x ^ (int(t) & 0xFFFFFFFF))
+    return x
 
 
 def blocks_for(num_tokens: int) -> int:
@@ -63,10 +90,17 @@ class OracleBlockManager:
         self.refcount = [0] * num_blocks
         self.tables: dict[int, list[int]] = {}
         self.lens: dict[int, int] = {}
+        # prefix caching ("PagedAttention与Continuous Batching原理与实践" §3.4,
+        # --enable-prefix-caching: a common prompt prefix is not recomputed)
+        self.prefix_caching = False
+        self.block_hash: dict[int, int] = {}   # block -> chained hash
+        self.valid: set[int] = set()           # hashed blocks whose KV was written
+        self.cache: dict[int, int] = {}        # hash -> block
+        self.evictable: OrderedDict[int, None] = OrderedDict()  # refcount-0 cached, oldest first
 
     # -- queries -----------------------------------------------------------
     def num_free(self) -> int:
-        return len(self.free_list)
+        return len(self.free_list) + len(self.evictable)
 
     def table(self, seq: int) -> list[int]:
         self._need(seq)
@@ -92,9 +126,9 @@ class OracleBlockManager:
         if num_tokens < 0:
             raise BMError("INVALID_ARG", "negative token count")
         n = blocks_for(num_tokens)
-        if n > len(self.free_list):
-            raise BMError("NO_BLOCKS", f"need {n}, have {len(self.free_list)}")
-        blocks = [self.free_list.popleft() for _ in range(n)]
+        if n > self.num_free():
+            raise BMError("NO_BLOCKS", f"need {n}, have {self.num_free()}")
+        blocks = [self._take_fresh() for _ in range(n)]
         for blk in blocks:
             self.refcount[blk] = 1
         self.tables[seq] = blocks
@@ -110,17 +144,17 @@ class OracleBlockManager:
         cow_src = cow_dst = -1
         if row == 0:
             # every page is full (or there is none): open a fresh page
-            if not self.free_list:
+            if not self.num_free():
                 raise BMError("NO_BLOCKS", "no block for a new page")
-            blk = self.free_list.popleft()
+            blk = self._take_fresh()
             self.refcount[blk] = 1
             tab.append(blk)
         else:
             last = tab[-1]
             if self.refcount[last] > 1:
-                if not self.free_list:
+                if not self.num_free():
                     raise BMError("NO_BLOCKS", "no block for copy-on-write")
-                blk = self.free_list.popleft()
+                blk = self._take_fresh()
                 self.refcount[blk] = 1
                 self.refcount[last] -= 1
                 tab[-1] = blk
@@ -145,8 +179,98 @@ class OracleBlockManager:
         for blk in self.tables.pop(seq):
             self.refcount[blk] -= 1
             if self.refcount[blk] == 0:
-                self.free_list.append(blk)
+                self._release(blk)
         del self.lens[seq]
+
+    # -- prefix caching -----------------------------------------------------
+    def set_prefix_caching(self, enable: bool) -> None:
+        if self.tables or len(self.free_list) != self.num_blocks:
+            raise BMError("INVALID_ARG", "only on a fresh block manager")
+        self.prefix_caching = bool(enable)
+
+    def allocate_prefix(self, seq: int, prompt_tokens, num_tokens: int) -> int:
+        """allocate() that shares the longest run of cached leading full blocks
+        of the prompt; returns the number of leading tokens whose KV is already
+        written (16 x the leading shared blocks that are valid)."""
+        if not self.prefix_caching:
+            self.allocate(seq, num_tokens)
+            return 0
+        if seq in self.tables:
+            raise BMError("SEQ_EXISTS", str(seq))
+        prompt = list(prompt_tokens)
+        if num_tokens < len(prompt):
+            raise BMError("INVALID_ARG", "fewer tokens than the prompt")
+        full = len(prompt) // BLOCK_SIZE
+        hashes, parent = [], 0
+        for i in range(full):
+            parent = chain_hash(parent, prompt[i * BLOCK_SIZE:(i + 1) * BLOCK_SIZE])
+            hashes.append(parent)
+        hits = []
+        for h in hashes:
+            if h not in self.cache:
+                break
+            hits.append(self.cache[h])
+        valid_prefix = 0
+        for blk in hits:
+            if blk not in self.valid:
+                break
+            valid_prefix += 1
+        total = blocks_for(num_tokens)
+        fresh = total - len(hits)
+        reused_free = sum(1 for blk in hits if self.refcount[blk] == 0)
+        if fresh > self.num_free() - reused_free:
+            raise BMError("NO_BLOCKS", f"need {fresh} new blocks")
+        table = []
+        for blk in hits:
+            if self.refcount[blk] == 0:
+                del self.evictable[blk]
+            self.refcount[blk] += 1
+            table.append(blk)
+        for i in range(len(hits), total):
+            blk = self._take_fresh()
+            self.refcount[blk] = 1
+            table.append(blk)
+            if i < full:
+                old = self.cache.get(hashes[i])
+                if old is not None:          # an unreachable leftover loses its entry
+                    self.block_hash.pop(old, None)
+                    self.valid.discard(old)
+                self.cache[hashes[i]] = blk
+                self.block_hash[blk] = hashes[i]
+                self.valid.discard(blk)
+        self.tables[seq] = table
+        self.lens[seq] = num_tokens
+        return valid_prefix * BLOCK_SIZE
+
+    def mark_written(self, seq: int) -> None:
+        self._need(seq)
+        for blk in self.tables[seq]:
+            if blk in self.block_hash:
+                self.valid.add(blk)
+
+    def _unregister(self, blk: int) -> None:
+        h = self.block_hash.pop(blk, None)
+        if h is not None and self.cache.get(h) == blk:
+            del self.cache[h]
+        self.valid.discard(blk)
+
+    def _take_fresh(self) -> int:
+        """A block for new content: the free list's head, else the least
+        recently released cached block (evicted)."""
+        if self.free_list:
+            return self.free_list.popleft()
+        blk, _ = self.evictable.popitem(last=False)
+        self._unregister(blk)
+        return blk
+
+    def _release(self, blk: int) -> None:
+        """Refcount of blk reached 0: a written cached block stays findable on
+        the evictable list; anything else returns to the free list."""
+        if blk in self.block_hash and blk in self.valid:
+            self.evictable[blk] = None
+        else:
+            self._unregister(blk)
+            self.free_list.append(blk)
 
     def _need(self, seq: int) -> None:
         if seq not in self.tables:

@@ -31,7 +31,11 @@ Readings where the pages are silent or loose (listed in the design notes):
     the grow phase ends (an error if nothing else is running: the pool cannot
     hold that request);
   * prompt K/V is (re)written only for requests admitted this step that are
-    still running at its end.
+    still running at its end;
+  * with prompt token ids (prefix caching), admission allocates through the
+    block manager's prefix cache and the prompt K/V is written from the first
+    position not covered by already-written cached blocks; the blocks of
+    requests admitted this step become reusable at its end.
 """
 from __future__ import annotations
 
@@ -64,6 +68,14 @@ class OracleScheduler:
         self.running: list[int] = []
         self.n_finished = 0
         self.step_idx = 0
+        self.tokens = None   # per-request prompt token ids when prefix caching is used
+
+    def set_prompt_tokens(self, tokens) -> None:
+        """Prompt token ids per request; admission then reuses cached prompt
+        blocks (the block manager's prefix caching must be on)."""
+        if self.step_idx != 0 or not self.bm.prefix_caching:
+            raise BMError("INVALID_ARG", "before the first step, with prefix caching on")
+        self.tokens = [list(t)[:self.prompt[i]] for i, t in enumerate(tokens)]
 
     def step(self) -> dict:
         s = self.step_idx
@@ -86,18 +98,29 @@ class OracleScheduler:
         # 3. admit from the head while its pages fit
         admitted = []
         admit_len = {}
+        admit_start = {}
         while self.waiting:
             r = self.waiting[0]
             total = self.prompt[r] + self.generated[r]
-            if blocks_for(total) > bm.num_free():
+            try:
+                if self.tokens is None:
+                    if blocks_for(total) > bm.num_free():
+                        raise BMError("NO_BLOCKS", "")
+                    bm.allocate(r, total)
+                    start = 0
+                else:
+                    start = bm.allocate_prefix(r, self.tokens[r], total)
+            except BMError as e:
+                if e.status != "NO_BLOCKS":
+                    raise
                 if not self.running:
                     raise BMError("NO_BLOCKS", f"request {r} can never fit")
                 break
             self.waiting.popleft()
-            bm.allocate(r, total)
             self.running.append(r)
             admitted.append(r)
             admit_len[r] = total
+            admit_start[r] = start
 
         # 4. grow every running request by one slot, preempting from the tail
         decode_slot = {}
@@ -135,7 +158,9 @@ class OracleScheduler:
         prompt_seqs = [r for r in admitted if r in still]
         prompt_slots = []
         for r in prompt_seqs:
-            prompt_slots.extend(bm.slots(r, 0, admit_len[r]))
+            prompt_slots.extend(bm.slots(r, admit_start[r], admit_len[r] - admit_start[r]))
+            if self.tokens is not None:
+                bm.mark_written(r)   # this step writes its KV: its cached blocks become reusable
         tables = []
         for r in running:
             tab = bm.table(r)
@@ -155,6 +180,8 @@ class OracleScheduler:
             "decode_slots": [decode_slot[r] for r in running],
             "prompt_seqs": prompt_seqs,
             "prompt_lens": [admit_len[r] for r in prompt_seqs],
+            "prompt_starts": [admit_start[r] for r in prompt_seqs],
+            "num_cached_tokens": sum(admit_start[r] for r in prompt_seqs),
             "prompt_slots": prompt_slots,
             "cow": cow,
             "admitted": admitted,

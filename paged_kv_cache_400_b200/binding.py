@@ -55,6 +55,7 @@ class pa_step_out(C.Structure):
         ("num_preempted", C.c_int32), ("preempted", _P64),
         ("num_finished", C.c_int32), ("finished", _P64),
         ("num_waiting", C.c_int32), ("num_free_blocks", C.c_int32),
+        ("prompt_starts", _P32), ("num_cached_tokens", C.c_int32),
     ]
 
 
@@ -92,6 +93,12 @@ def _declare(lib):
         "pa_sched_create": (i32, [vp, _P32, _P32, _P32, i32, i32, C.POINTER(vp)]),
         "pa_sched_step": (i32, [vp, C.POINTER(pa_step_out)]),
         "pa_sched_destroy": (None, [vp]),
+        "pa_sched_set_prompt_tokens": (i32, [vp, _P32, _P64]),
+        "pa_bm_set_prefix_caching": (i32, [vp, i32]),
+        "pa_bm_allocate_prefix": (i32, [vp, i64, _P32, i32, i32, _P32]),
+        "pa_bm_mark_written": (i32, [vp, i64]),
+        "pa_bm_evictable_list": (i32, [vp, _P32, i32, _P32]),
+        "pa_bm_num_cached": (i32, [vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -348,6 +355,30 @@ class BlockManager:
         _check("pa_bm_free_list", lib().pa_bm_free_list(self.handle, _i32p(buf), self.num_blocks, C.byref(n)))
         return buf[: n.value].tolist()
 
+    def set_prefix_caching(self, enable: bool):
+        _check("pa_bm_set_prefix_caching", lib().pa_bm_set_prefix_caching(self.handle, int(bool(enable))))
+
+    def allocate_prefix(self, seq: int, prompt_tokens, num_tokens: int) -> int:
+        """Allocation sharing cached prompt blocks; returns the cached tokens."""
+        toks = np.ascontiguousarray(prompt_tokens, dtype=np.int32)
+        cached = C.c_int32()
+        _check("pa_bm_allocate_prefix", lib().pa_bm_allocate_prefix(
+            self.handle, seq, _i32p(toks), len(toks), num_tokens, C.byref(cached)))
+        return cached.value
+
+    def mark_written(self, seq: int):
+        _check("pa_bm_mark_written", lib().pa_bm_mark_written(self.handle, seq))
+
+    def evictable_list(self) -> list:
+        n = C.c_int32()
+        buf = np.empty(self.num_blocks, dtype=np.int32)
+        _check("pa_bm_evictable_list", lib().pa_bm_evictable_list(self.handle, _i32p(buf), self.num_blocks,
+                                                                  C.byref(n)))
+        return buf[: n.value].tolist()
+
+    def num_cached(self) -> int:
+        return int(lib().pa_bm_num_cached(self.handle))
+
     def slots(self, seq: int, start: int, count: int) -> np.ndarray:
         out = np.empty(count, dtype=np.int64)
         _check("pa_bm_slots", lib().pa_bm_slots(self.handle, seq, start, count, _i64p(out)))
@@ -391,6 +422,15 @@ class Scheduler:
         except Exception:
             pass
 
+    def set_prompt_tokens(self, tokens):
+        """Per-request prompt token ids (prefix-cached admission)."""
+        lens = [len(t) for t in tokens]
+        flat = np.ascontiguousarray(np.concatenate([np.asarray(t, np.int32) for t in tokens])
+                                    if tokens else np.zeros(0, np.int32), dtype=np.int32)
+        offs = np.ascontiguousarray(np.concatenate([[0], np.cumsum(lens)[:-1]]), dtype=np.int64)
+        _check("pa_sched_set_prompt_tokens", lib().pa_sched_set_prompt_tokens(self.handle, _i32p(flat),
+                                                                              _i64p(offs)))
+
     def step_raw(self) -> pa_step_out:
         """Runs one step; the returned struct's arrays are valid until the next."""
         _check("pa_sched_step", lib().pa_sched_step(self.handle, C.byref(self._out)))
@@ -422,6 +462,8 @@ class Scheduler:
             "preempted": arr(o.preempted, o.num_preempted, np.int64),
             "finished": arr(o.finished, o.num_finished, np.int64),
             "num_waiting": o.num_waiting, "num_free_blocks": o.num_free_blocks,
+            "prompt_starts": arr(o.prompt_starts, o.num_prompt_seqs, np.int32),
+            "num_cached_tokens": o.num_cached_tokens,
         }
 
 

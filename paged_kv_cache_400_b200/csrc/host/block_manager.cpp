@@ -61,6 +61,12 @@ pa_status pa_bm_create(int32_t num_blocks, int32_t block_size,
   }
   bm->head = 0;
   bm->count = num_blocks;
+  bm->block_hash.assign(num_blocks, 0);
+  bm->has_hash.assign(num_blocks, 0);
+  bm->valid.assign(num_blocks, 0);
+  bm->ev_prev.assign(num_blocks, -1);
+  bm->ev_next.assign(num_blocks, -1);
+  bm->in_ev.assign(num_blocks, 0);
   *out = bm;
   return PA_OK;
 }
@@ -72,12 +78,12 @@ pa_status pa_bm_allocate(pa_bm* bm, int64_t seq, int32_t num_tokens) {
   if (num_tokens < 0) return fail(PA_ERR_INVALID_ARG, "pa_bm_allocate: num_tokens %d", num_tokens);
   if (bm->seqs.count(seq)) return fail(PA_ERR_SEQ_EXISTS, "pa_bm_allocate: seq %lld exists", (long long)seq);
   const int32_t n = pagedkv::blocks_for(num_tokens);
-  if (n > bm->count)
-    return fail(PA_ERR_NO_BLOCKS, "pa_bm_allocate: need %d blocks, %d free", n, bm->count);
+  if (n > bm->free_blocks())
+    return fail(PA_ERR_NO_BLOCKS, "pa_bm_allocate: need %d blocks, %d free", n, bm->free_blocks());
   pagedkv::SeqState st;
   st.table.reserve(n + 1);
   for (int32_t i = 0; i < n; ++i) {
-    int32_t b = bm->pop_front();
+    int32_t b = bm->take_fresh();
     bm->refcount[b] = 1;
     st.table.push_back(b);
   }
@@ -99,16 +105,16 @@ pa_status pa_bm_append_slot(pa_bm* bm, int64_t seq, int64_t* slot, int32_t* cow_
   int32_t cs = -1, cd = -1;
   if (row == 0) {
     // every page is full (or there is none): a fresh page
-    if (bm->count == 0) return fail(PA_ERR_NO_BLOCKS, "pa_bm_append_slot: no free block");
-    blk = bm->pop_front();
+    if (bm->free_blocks() == 0) return fail(PA_ERR_NO_BLOCKS, "pa_bm_append_slot: no free block");
+    blk = bm->take_fresh();
     bm->refcount[blk] = 1;
     st.table.push_back(blk);
   } else {
     const int32_t last = st.table.back();
     if (bm->refcount[last] > 1) {
       // shared partial page: copy-on-write
-      if (bm->count == 0) return fail(PA_ERR_NO_BLOCKS, "pa_bm_append_slot: no block for copy-on-write");
-      blk = bm->pop_front();
+      if (bm->free_blocks() == 0) return fail(PA_ERR_NO_BLOCKS, "pa_bm_append_slot: no block for copy-on-write");
+      blk = bm->take_fresh();
       bm->refcount[blk] = 1;
       bm->refcount[last] -= 1;
       st.table.back() = blk;
@@ -141,13 +147,13 @@ pa_status pa_bm_free(pa_bm* bm, int64_t seq) {
   auto it = bm->seqs.find(seq);
   if (it == bm->seqs.end()) return fail(PA_ERR_UNKNOWN_SEQ, "pa_bm_free: seq %lld", (long long)seq);
   for (int32_t b : it->second.table) {
-    if (--bm->refcount[b] == 0) bm->push_back(b);
+    if (--bm->refcount[b] == 0) bm->release(b);
   }
   bm->seqs.erase(it);
   return PA_OK;
 }
 
-int32_t pa_bm_num_free(const pa_bm* bm) { return bm ? bm->count : 0; }
+int32_t pa_bm_num_free(const pa_bm* bm) { return bm ? bm->free_blocks() : 0; }
 int32_t pa_bm_num_blocks(const pa_bm* bm) { return bm ? bm->num_blocks : 0; }
 
 pa_status pa_bm_seq_len(const pa_bm* bm, int64_t seq, int32_t* len) {
@@ -201,6 +207,98 @@ pa_status pa_bm_slots(const pa_bm* bm, int64_t seq, int32_t start, int32_t count
   }
   return PA_OK;
 }
+
+pa_status pa_bm_set_prefix_caching(pa_bm* bm, int32_t enable) {
+  if (!bm) return fail(PA_ERR_INVALID_ARG, "pa_bm_set_prefix_caching: bm is NULL");
+  if (!bm->seqs.empty() || bm->count != bm->num_blocks)
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_set_prefix_caching: only on a fresh block manager");
+  bm->prefix_caching = enable != 0;
+  return PA_OK;
+}
+
+pa_status pa_bm_allocate_prefix(pa_bm* bm, int64_t seq, const int32_t* prompt_tokens,
+                                int32_t num_prompt_tokens, int32_t num_tokens, int32_t* cached_tokens) {
+  if (!bm || !cached_tokens || (num_prompt_tokens > 0 && !prompt_tokens))
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_allocate_prefix: NULL argument");
+  if (num_prompt_tokens < 0 || num_tokens < num_prompt_tokens)
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_allocate_prefix: %d prompt tokens, %d tokens", num_prompt_tokens,
+                num_tokens);
+  if (bm->seqs.count(seq))
+    return fail(PA_ERR_SEQ_EXISTS, "pa_bm_allocate_prefix: seq %lld exists", (long long)seq);
+  *cached_tokens = 0;
+  if (!bm->prefix_caching) return pa_bm_allocate(bm, seq, num_tokens);
+  const int32_t total = pagedkv::blocks_for(num_tokens);
+  const int32_t full = num_prompt_tokens / PA_BLOCK_SIZE;
+  std::vector<uint64_t> h(full);
+  uint64_t parent = 0;
+  for (int32_t i = 0; i < full; ++i) parent = h[i] = pagedkv::chain_hash(parent, prompt_tokens + i * PA_BLOCK_SIZE);
+  // longest run of cached leading blocks
+  std::vector<int32_t> hits;
+  int32_t hits_evictable = 0, valid_prefix = 0;
+  bool all_valid = true;
+  for (int32_t i = 0; i < full; ++i) {
+    auto it = bm->cache.find(h[i]);
+    if (it == bm->cache.end()) break;
+    const int32_t b = it->second;
+    hits.push_back(b);
+    if (bm->refcount[b] == 0) ++hits_evictable;
+    if (all_valid && bm->valid[b]) ++valid_prefix;
+    else all_valid = false;
+  }
+  const int32_t fresh = total - (int32_t)hits.size();
+  if (fresh > bm->free_blocks() - hits_evictable)
+    return fail(PA_ERR_NO_BLOCKS, "pa_bm_allocate_prefix: need %d new blocks, %d free (%d of them reused)", fresh,
+                bm->free_blocks(), hits_evictable);
+  pagedkv::SeqState st;
+  st.table.reserve(total + 1);
+  for (int32_t b : hits) {
+    if (bm->refcount[b] == 0) bm->ev_remove(b);
+    bm->refcount[b] += 1;
+    st.table.push_back(b);
+  }
+  for (int32_t i = (int32_t)hits.size(); i < total; ++i) {
+    const int32_t b = bm->take_fresh();
+    bm->refcount[b] = 1;
+    st.table.push_back(b);
+    if (i < full) {
+      // a new full prompt block: cached under its chain hash, valid once written
+      auto it = bm->cache.find(h[i]);
+      if (it != bm->cache.end()) {  // an unreachable leftover loses its entry
+        bm->has_hash[it->second] = 0;
+        bm->valid[it->second] = 0;
+      }
+      bm->cache[h[i]] = b;
+      bm->block_hash[b] = h[i];
+      bm->has_hash[b] = 1;
+      bm->valid[b] = 0;
+    }
+  }
+  st.len = num_tokens;
+  bm->seqs.emplace(seq, std::move(st));
+  *cached_tokens = valid_prefix * PA_BLOCK_SIZE;
+  return PA_OK;
+}
+
+pa_status pa_bm_mark_written(pa_bm* bm, int64_t seq) {
+  if (!bm) return fail(PA_ERR_INVALID_ARG, "pa_bm_mark_written: bm is NULL");
+  auto it = bm->seqs.find(seq);
+  if (it == bm->seqs.end()) return fail(PA_ERR_UNKNOWN_SEQ, "pa_bm_mark_written: seq %lld", (long long)seq);
+  for (int32_t b : it->second.table)
+    if (bm->has_hash[b]) bm->valid[b] = 1;
+  return PA_OK;
+}
+
+pa_status pa_bm_evictable_list(const pa_bm* bm, int32_t* out, int32_t cap, int32_t* n) {
+  if (!bm || !n || (cap > 0 && !out) || cap < 0)
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_evictable_list: bad argument");
+  *n = bm->ev_count;
+  if (bm->ev_count > cap) return fail(PA_ERR_CAPACITY, "pa_bm_evictable_list: %d > cap %d", bm->ev_count, cap);
+  int32_t i = 0;
+  for (int32_t b = bm->ev_head; b >= 0; b = bm->ev_next[b]) out[i++] = b;
+  return PA_OK;
+}
+
+int32_t pa_bm_num_cached(const pa_bm* bm) { return bm ? (int32_t)bm->cache.size() : 0; }
 
 pa_status pa_bm_pack(const pa_bm* bm, const int64_t* seqs, int32_t n, int32_t max_blocks,
                      int32_t* block_tables, int32_t* seq_lens, int64_t* last_slots) {

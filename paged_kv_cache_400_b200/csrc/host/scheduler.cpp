@@ -34,12 +34,16 @@ struct pa_sched {
   std::vector<int64_t> running;
   std::vector<char> is_running;
   std::vector<int32_t> admit_len;
+  std::vector<int32_t> admit_start;         // first position whose KV the admission writes
+  std::vector<int32_t> tokens;              // prompt token ids (prefix caching), or empty
+  std::vector<int64_t> token_offset;        // request i's prompt: tokens[token_offset[i] ...]
   int32_t n_finished = 0;
   int32_t step_idx = 0;
   // step outputs
   std::vector<int64_t> o_running, o_decode_slots, o_prompt_seqs, o_prompt_slots;
   std::vector<int64_t> o_admitted, o_preempted, o_finished;
-  std::vector<int32_t> o_seq_lens, o_block_tables, o_prompt_lens, o_cow_src, o_cow_dst;
+  std::vector<int32_t> o_seq_lens, o_block_tables, o_prompt_lens, o_cow_src, o_cow_dst, o_prompt_starts;
+  int32_t o_cached_tokens = 0;
   std::vector<int64_t> slot_of;  // per request: slot appended this step
 };
 
@@ -67,7 +71,9 @@ void publish(pa_sched* s, pa_step_out* out) {
   out->num_finished = (int32_t)s->o_finished.size();
   out->finished = s->o_finished.data();
   out->num_waiting = (int32_t)s->waiting.size();
-  out->num_free_blocks = s->bm->count;
+  out->num_free_blocks = s->bm->free_blocks();
+  out->prompt_starts = s->o_prompt_starts.data();
+  out->num_cached_tokens = s->o_cached_tokens;
 }
 
 }  // namespace
@@ -100,6 +106,7 @@ pa_status pa_sched_create(pa_bm* bm, const int32_t* arrival_step, const int32_t*
   s->generated.assign(n_requests, 0);
   s->is_running.assign(n_requests, 0);
   s->admit_len.assign(n_requests, 0);
+  s->admit_start.assign(n_requests, 0);
   s->slot_of.assign(n_requests, -1);
   s->arrival_order.resize(n_requests);
   std::iota(s->arrival_order.begin(), s->arrival_order.end(), 0);
@@ -110,6 +117,21 @@ pa_status pa_sched_create(pa_bm* bm, const int32_t* arrival_step, const int32_t*
 }
 
 void pa_sched_destroy(pa_sched* s) { delete s; }
+
+pa_status pa_sched_set_prompt_tokens(pa_sched* s, const int32_t* tokens, const int64_t* offsets) {
+  if (!s || !tokens || !offsets) return fail(PA_ERR_INVALID_ARG, "pa_sched_set_prompt_tokens: NULL argument");
+  if (s->step_idx != 0) return fail(PA_ERR_INVALID_ARG, "pa_sched_set_prompt_tokens: only before the first step");
+  if (!s->bm->prefix_caching)
+    return fail(PA_ERR_INVALID_ARG, "pa_sched_set_prompt_tokens: the block manager's prefix caching is off");
+  int64_t end = 0;
+  for (int32_t i = 0; i < s->n; ++i) {
+    if (offsets[i] < 0) return fail(PA_ERR_INVALID_ARG, "pa_sched_set_prompt_tokens: offset %d", i);
+    end = std::max(end, offsets[i] + s->prompt[i]);
+  }
+  s->tokens.assign(tokens, tokens + end);
+  s->token_offset.assign(offsets, offsets + s->n);
+  return PA_OK;
+}
 
 pa_status pa_sched_step(pa_sched* s, pa_step_out* out) {
   if (!s || !out) return fail(PA_ERR_INVALID_ARG, "pa_sched_step: NULL argument");
@@ -127,6 +149,8 @@ pa_status pa_sched_step(pa_sched* s, pa_step_out* out) {
   s->o_prompt_lens.clear();
   s->o_cow_src.clear();
   s->o_cow_dst.clear();
+  s->o_prompt_starts.clear();
+  s->o_cached_tokens = 0;
   out->step = step;
 
   // 1. retire requests that generated all their tokens; pages return at once
@@ -153,23 +177,32 @@ pa_status pa_sched_step(pa_sched* s, pa_step_out* out) {
     ++s->next_arrival;
   }
 
-  // 3. admit from the head while its pages fit (first come, first served)
+  // 3. admit from the head while its pages fit (first come, first served);
+  //    with prompt tokens, the cached leading blocks of the prompt are reused
+  //    and only the rest of its KV is (re)written
   while (!s->waiting.empty()) {
     const int64_t r = s->waiting.front();
     const int32_t total = s->prompt[r] + s->generated[r];
-    if (pagedkv::blocks_for(total) > bm->count) {
+    int32_t cached = 0;
+    pa_status st;
+    if (s->tokens.empty()) {
+      st = pagedkv::blocks_for(total) > bm->free_blocks() ? PA_ERR_NO_BLOCKS : pa_bm_allocate(bm, r, total);
+    } else {
+      st = pa_bm_allocate_prefix(bm, r, s->tokens.data() + s->token_offset[r], s->prompt[r], total, &cached);
+    }
+    if (st == PA_ERR_NO_BLOCKS) {
       if (s->running.empty())
         return fail(PA_ERR_NO_BLOCKS, "pa_sched_step: request %lld can never fit (%d tokens, %d blocks)",
                     (long long)r, total, bm->num_blocks);
       break;
     }
-    s->waiting.pop_front();
-    pa_status st = pa_bm_allocate(bm, r, total);
     if (st != PA_OK) return st;
+    s->waiting.pop_front();
     s->running.push_back(r);
     s->is_running[r] = 1;
     s->o_admitted.push_back(r);
     s->admit_len[r] = total;
+    s->admit_start[r] = cached;
   }
 
   // 4. grow every running request by one slot; preempt the newest on shortage
@@ -221,12 +254,17 @@ pa_status pa_sched_step(pa_sched* s, pa_step_out* out) {
   for (int64_t r : s->o_admitted) {
     if (!s->is_running[r]) continue;  // admitted, then preempted in the same step
     const int32_t n = s->admit_len[r];
+    const int32_t start = s->admit_start[r];
     s->o_prompt_seqs.push_back(r);
     s->o_prompt_lens.push_back(n);
+    s->o_prompt_starts.push_back(start);
+    s->o_cached_tokens += start;
     const size_t at = s->o_prompt_slots.size();
-    s->o_prompt_slots.resize(at + n);
-    pa_status st = pa_bm_slots(bm, r, 0, n, s->o_prompt_slots.data() + at);
+    s->o_prompt_slots.resize(at + (n - start));
+    pa_status st = pa_bm_slots(bm, r, start, n - start, s->o_prompt_slots.data() + at);
     if (st != PA_OK) return st;
+    // this step's device work writes its KV: its cached blocks become reusable
+    if (!s->tokens.empty() && (st = pa_bm_mark_written(bm, r)) != PA_OK) return st;
   }
 
   // 6. every running request generated one token

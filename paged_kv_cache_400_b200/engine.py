@@ -46,6 +46,7 @@ class StepIndices:
     decode_slots: np.ndarray
     prompt_seqs: np.ndarray
     prompt_lens: np.ndarray
+    prompt_starts: np.ndarray
     prompt_slots: np.ndarray
     cow_src: np.ndarray
     cow_dst: np.ndarray
@@ -56,7 +57,10 @@ class StepIndices:
 class DecodeEngine:
     def __init__(self, num_blocks, num_layers, num_heads, num_kv_heads, head_dim, arrival_step,
                  prompt_len, output_len, table_width, scale, device, dtype=torch.bfloat16,
-                 max_seq_len=None):
+                 max_seq_len=None, prompt_tokens=None):
+        """prompt_tokens: per-request prompt token ids to turn on automatic
+        prefix caching (admission reuses cached prompt blocks and only the KV
+        after the cached prefix is written)."""
         self.device = torch.device(device)
         self.num_layers = num_layers
         self.num_heads = num_heads
@@ -66,7 +70,11 @@ class DecodeEngine:
         self.table_width = table_width
         self.max_seq_len = max_seq_len or table_width * bd.BLOCK_SIZE
         self.bm = bd.BlockManager(num_blocks)
+        if prompt_tokens is not None:
+            self.bm.set_prefix_caching(True)
         self.sched = bd.Scheduler(self.bm, arrival_step, prompt_len, output_len, table_width)
+        if prompt_tokens is not None:
+            self.sched.set_prompt_tokens(prompt_tokens)
         shape = (num_blocks, 2, num_kv_heads, bd.BLOCK_SIZE, head_dim)
         self.pools = [torch.empty(shape, dtype=dtype, device=self.device) for _ in range(num_layers)]
         self._ws = None
@@ -98,6 +106,7 @@ class DecodeEngine:
             decode_slots=arr(o.decode_slots, n, np.int64),
             prompt_seqs=arr(o.prompt_seqs, o.num_prompt_seqs, np.int64),
             prompt_lens=arr(o.prompt_lens, o.num_prompt_seqs, np.int32),
+            prompt_starts=arr(o.prompt_starts, o.num_prompt_seqs, np.int32),
             prompt_slots=arr(o.prompt_slots, o.num_prompt_tokens, np.int64),
             cow_src=arr(o.cow_src, o.num_cow, np.int32),
             cow_dst=arr(o.cow_dst, o.num_cow, np.int32),
@@ -110,10 +119,12 @@ class DecodeEngine:
 
     @staticmethod
     def prompt_positions(idx: StepIndices):
-        """(request, position) of every prompt slot, in prompt_slots order."""
-        reqs = np.repeat(idx.prompt_seqs, idx.prompt_lens)
-        pos = np.concatenate([np.arange(n) for n in idx.prompt_lens]) if len(idx.prompt_lens) else \
-            np.empty(0, np.int64)
+        """(request, position) of every prompt slot, in prompt_slots order
+        (positions start..len-1 of each admitted request)."""
+        counts = idx.prompt_lens - idx.prompt_starts
+        reqs = np.repeat(idx.prompt_seqs, counts)
+        pos = np.concatenate([np.arange(a, n) for a, n in zip(idx.prompt_starts, idx.prompt_lens)]) \
+            if len(idx.prompt_lens) else np.empty(0, np.int64)
         return reqs, pos
 
     # ---- device side -------------------------------------------------------------

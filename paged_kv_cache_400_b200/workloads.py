@@ -291,6 +291,22 @@ class TraceCase:
     dtype: str
     scale: float
     table_width: int
+    # shared-prompt traces: prompt token ids per request, and which of the
+    # system prompts (sys_id) covers its first sys_len tokens
+    prompt_tokens: list = None
+    sys_id: np.ndarray = None
+    sys_len: np.ndarray = None
+
+    def _owner(self, reqs: torch.Tensor, pos: torch.Tensor) -> torch.Tensor:
+        """Value stream of each (request, position): a system prompt's own
+        stream inside it (identical prefixes hold identical K/V, as a model's
+        would), the request's stream elsewhere."""
+        if self.sys_len is None:
+            return reqs
+        dev = reqs.device
+        sl = torch.as_tensor(self.sys_len, dtype=torch.int64, device=dev)[reqs]
+        sid = torch.as_tensor(self.sys_id, dtype=torch.int64, device=dev)[reqs]
+        return torch.where(pos < sl, TRACE_MAX_REQ + sid, reqs)
 
     def kv_values(self, layer: int, reqs, positions, device="cpu"):
         """K and V of token `positions[i]` of request `reqs[i]` in `layer`:
@@ -300,7 +316,7 @@ class TraceCase:
         per_tok = 2 * self.num_kv_heads * self.head_dim
         r = torch.as_tensor(np.asarray(reqs, dtype=np.int64), device=device)
         p = torch.as_tensor(np.asarray(positions, dtype=np.int64), device=device)
-        base = (r * TRACE_MAX_POS + p) * per_tok
+        base = (self._owner(r, p) * TRACE_MAX_POS + p) * per_tok
         c = base[:, None] + torch.arange(per_tok, device=device)[None, :]
         x = values(stream_key(self.seed, TAG_TRACE_KV, layer), c).to(TORCH_DTYPE[self.dtype])
         x = x.reshape(len(r), 2, self.num_kv_heads, self.head_dim)
@@ -327,7 +343,7 @@ class TraceCase:
                               dtype=torch.int64, device=device)[:, None]
         r = torch.as_tensor(np.asarray(running, np.int64), device=device)
         p = torch.as_tensor(dec_pos, device=device)
-        c = (((r * TRACE_MAX_POS + p) * per_tok)[:, None]
+        c = (((self._owner(r, p) * TRACE_MAX_POS + p) * per_tok)[:, None]
              + torch.arange(per_tok, device=device)[None, :]).reshape(1, -1)
         kv_all = values(kv_keys, c).to(dt).reshape(L, n, 2, self.num_kv_heads, self.head_dim)
         per_q = self.num_heads * self.head_dim
@@ -376,3 +392,33 @@ def trace_case(seed: int = 0, n_requests: int = 2000, rate: float = 50.0,
                      num_blocks=num_blocks, num_layers=num_layers, num_heads=32,
                      num_kv_heads=8, head_dim=128, dtype="bf16", scale=128 ** -0.5,
                      table_width=192)
+
+
+def prefix_trace_case(seed: int = 0, n_requests: int = 2000, rate: float = 50.0,
+                      num_blocks: int = 40000, num_layers: int = 32, n_system: int = 8,
+                      vocab: int = 32000) -> TraceCase:
+    """The arrival trace with shared prompts: every request's prompt is one of
+    `n_system` system prompts (length uniform in [256, 1024]) followed by its
+    own user tokens (length uniform in [16, 512]); token ids uniform in
+    [0, vocab). Arrivals and output lengths as in trace_case."""
+    rng = np.random.default_rng(seed + 606)
+    arrivals = []
+    step = 0
+    while len(arrivals) < n_requests:
+        arrivals.extend([step] * int(rng.poisson(rate)))
+        step += 1
+    arrivals = np.asarray(arrivals[:n_requests], dtype=np.int32)
+    systems = [rng.integers(0, vocab, size=int(rng.integers(256, 1024, endpoint=True))).astype(np.int32)
+               for _ in range(n_system)]
+    sys_id = rng.integers(0, n_system, size=n_requests).astype(np.int32)
+    prompts = []
+    for i in range(n_requests):
+        user = rng.integers(0, vocab, size=int(rng.integers(16, 512, endpoint=True))).astype(np.int32)
+        prompts.append(np.concatenate([systems[sys_id[i]], user]))
+    prompt_len = np.asarray([len(p) for p in prompts], dtype=np.int32)
+    output = np.minimum(rng.geometric(1.0 / 200.0, size=n_requests), 2048).astype(np.int32)
+    sys_len = np.asarray([len(systems[s]) for s in sys_id], dtype=np.int32)
+    return TraceCase(seed=seed, arrival_step=arrivals, prompt_len=prompt_len, output_len=output,
+                     num_blocks=num_blocks, num_layers=num_layers, num_heads=32, num_kv_heads=8,
+                     head_dim=128, dtype="bf16", scale=128 ** -0.5, table_width=224,
+                     prompt_tokens=prompts, sys_id=sys_id, sys_len=sys_len)

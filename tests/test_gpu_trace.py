@@ -130,3 +130,49 @@ def test_graphed_layer_loop_matches_oracle():
     assert pk.pa_get_device_error() == 0
     assert checked >= 10 and len(graphed.graphs) >= 2
     eng.close()
+
+
+def test_shared_prompt_trace_with_prefix_caching_matches_oracle():
+    """Requests share system prompts; with prefix caching their full system
+    prompt blocks are reused and never rewritten. Each sampled output must
+    still equal the oracle's attention over the request's whole prompt."""
+    trace = wl.prefix_trace_case(seed=7, n_requests=160, rate=12.0, num_blocks=2600, num_layers=2,
+                                 n_system=3)
+    trace.output_len = np.minimum(trace.output_len, 150).astype(np.int32)
+    eng = DecodeEngine(trace.num_blocks, trace.num_layers, trace.num_heads, trace.num_kv_heads,
+                       trace.head_dim, trace.arrival_step, trace.prompt_len, trace.output_len,
+                       trace.table_width, trace.scale, DEV, prompt_tokens=trace.prompt_tokens)
+    obm = OracleBlockManager(trace.num_blocks)
+    obm.set_prefix_caching(True)
+    osch = OracleScheduler(obm, trace.arrival_step, trace.prompt_len, trace.output_len, trace.table_width)
+    osch.set_prompt_tokens(trace.prompt_tokens)
+    rng = np.random.default_rng(2)
+    checked = hits_checked = cached_total = 0
+    started_cached = set()
+    while True:
+        idx = eng.schedule()
+        o = osch.step()
+        assert idx.prompt_slots.tolist() == o["prompt_slots"]
+        assert idx.prompt_starts.tolist() == o["prompt_starts"]
+        cached_total += int(idx.prompt_starts.sum())
+        started_cached.update(int(r) for r, a in zip(idx.prompt_seqs, idx.prompt_starts) if a > 0)
+        if len(idx.running):
+            inputs = [layer_inputs(trace, eng, idx, l, DEV) for l in range(trace.num_layers)]
+            outs = eng.run_layers(idx, inputs)
+            if idx.step % 7 == 0 and checked < 40:
+                layer = int(rng.integers(0, trace.num_layers))
+                got = outs[layer].float().cpu().numpy()
+                for i in rng.choice(len(idx.running), size=min(3, len(idx.running)), replace=False):
+                    r = int(idx.running[i])
+                    ref = oracle_attention(trace, layer, idx.step, r,
+                                           o["block_tables"][i][:(o["seq_lens"][i] + 15) // 16],
+                                           o["seq_lens"][i])
+                    assert float(np.abs(got[i] - ref).max()) <= 1e-2, (idx.step, r)
+                    checked += 1
+                    hits_checked += r in started_cached
+        if idx.done:
+            break
+    import paged_kv_cache_400_b200 as pk
+    assert pk.pa_get_device_error() == 0
+    assert cached_total > 0 and hits_checked >= 5 and checked >= 20, (cached_total, hits_checked, checked)
+    eng.close()
