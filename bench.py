@@ -51,6 +51,8 @@ def parse_args():
                     help="gqa is the benchmark line; the others are extra measurements")
     ap.add_argument("--trace-layers", type=int, default=32)
     ap.add_argument("--trace-requests", type=int, default=2000)
+    ap.add_argument("--swap-host-blocks", type=int, default=0,
+                    help="trace: pinned host blocks per layer for swap-mode preemption (0: recompute)")
     ap.add_argument("--no-prefix-cache", action="store_true",
                     help="prefix_trace: run without automatic prefix caching (for comparison)")
     ap.add_argument("--graphs", action="store_true",
@@ -497,7 +499,8 @@ def run_trace(args, rank, world):
     caching = shared and not args.no_prefix_cache
     eng = DecodeEngine(tr.num_blocks, tr.num_layers, tr.num_heads, tr.num_kv_heads, tr.head_dim,
                        tr.arrival_step, tr.prompt_len, tr.output_len, tr.table_width, tr.scale, dev,
-                       prompt_tokens=tr.prompt_tokens if caching else None)
+                       prompt_tokens=tr.prompt_tokens if caching else None,
+                       swap_host_blocks=args.swap_host_blocks)
     graphed = None
     if args.graphs:
         from paged_kv_cache_400_b200.engine import GraphedLayers
@@ -505,6 +508,7 @@ def run_trace(args, rank, world):
     stream = torch.cuda.current_stream()
     events = []
     tokens = kv_tokens = prompt_tokens = steps = preempted = cached_tokens = peak_batch = 0
+    swap_blocks = 0
     host_s = e2e_s = 0.0
     sampler = ClockSampler(local)
     sampler.start()
@@ -539,6 +543,7 @@ def run_trace(args, rank, world):
         steps += 1
         preempted += idx.record.preempted
         cached_tokens += int(idx.prompt_starts.sum())
+        swap_blocks += len(idx.swap_out) + len(idx.swap_in)
         peak_batch = max(peak_batch, n)
         if idx.done:
             break
@@ -558,6 +563,8 @@ def run_trace(args, rank, world):
                     f"{tr.num_layers} layers x (prompt append + decode-token append + paged decode), "
                     "32/8 heads, head_dim 128, bf16",
         "prompt_tokens_cached": cached_tokens, "peak_batch": peak_batch,
+        "swap_host_blocks": args.swap_host_blocks,
+        "swap_bytes": swap_blocks * 2 * tr.num_kv_heads * 16 * tr.head_dim * 2 * tr.num_layers,
         "metric": "generated tokens/s (device time of the layer loops)", "value": tokens / gpu_s,
         "unit": "tokens/s", "steps": steps, "generated_tokens": tokens, "prompt_tokens_written": prompt_tokens,
         "preemptions": preempted, "gpu_s": gpu_s, "host_scheduler_s": host_s,

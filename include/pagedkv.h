@@ -230,6 +230,21 @@ pa_status pa_copy_blocks(void* kv_pool, const int32_t* src, const int32_t* dst,
                          int32_t n, pa_pool_desc pool, void* stream);
 
 /*
+ * Block copy between two pools of the same block shape (pool's kv heads,
+ * head_dim, dtype): for i in [0, n), block src[i] of src_pool is copied to
+ * block dst[i] of dst_pool. Either pool may be device memory or pinned host
+ * memory mapped into the device's address space (e.g. from cudaHostAlloc),
+ * which is how swap-mode preemption moves a preempted sequence's blocks to
+ * host memory and back ([A] §3.4 "--swap-space"; [B] "Preemption（抢占）":
+ * swap the KV cache out to the CPU). src, dst: int32 [n] the GPU can read.
+ * Pointers the GPU cannot address are rejected (PA_ERR_INVALID_ARG) before
+ * any launch; an id outside its pool skips the pair and sets PA_DEVERR_BLOCK.
+ */
+pa_status pa_copy_blocks_between(void* dst_pool, int32_t dst_num_blocks, const void* src_pool,
+                                 int32_t src_num_blocks, const int32_t* src, const int32_t* dst,
+                                 int32_t n, pa_pool_desc pool, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's error
  * word (PA_DEVERR_* bits) into *flags. Returns PA_ERR_DEVICE_BOUNDS when the
  * word was non-zero, PA_OK when zero.
@@ -393,6 +408,20 @@ typedef struct {
                                    blocks (0 without prefix caching); the
                                    request's prompt_slots cover [start, len)  */
   int32_t num_cached_tokens;    /* sum of prompt_starts this step              */
+  /* swap-mode preemption (pa_sched_set_swap); device work order of a step:
+     swap-out copies, swap-in copies, copy-on-write copies, prompt appends,
+     decode */
+  int32_t num_swap_out;
+  const int32_t* swap_out_src;  /* [num_swap_out] device blocks to copy ...    */
+  const int32_t* swap_out_dst;  /* ... into these host blocks                  */
+  int32_t num_swap_in;
+  const int32_t* swap_in_src;   /* [num_swap_in] host blocks to copy ...       */
+  const int32_t* swap_in_dst;   /* ... into these device blocks                */
+  int32_t num_swapped_out;
+  const int64_t* swapped_out;   /* preempted this step by swapping out         */
+  int32_t num_swapped_in;
+  const int64_t* swapped_in;    /* admitted this step by swapping in (not in
+                                   prompt_seqs: nothing is recomputed)        */
 } pa_step_out;
 
 /*
@@ -437,6 +466,18 @@ pa_status pa_sched_step(pa_sched* s, pa_step_out* out);
  * the first step. Arrays are copied.
  */
 pa_status pa_sched_set_prompt_tokens(pa_sched* s, const int32_t* tokens, const int64_t* offsets);
+/*
+ * Swap-mode preemption ([B] "Preemption（抢占）": the second mode swaps the KV
+ * cache to the CPU; [A] §3.4 "--swap-space"). With num_host_blocks > 0 host
+ * blocks, a preemption victim whose KV was written before the step and whose
+ * blocks are not shared is swapped out: its blocks go to host blocks taken from
+ * a FIFO host free list (swap_out pairs) and, when it is admitted again, into
+ * fresh device blocks (swap_in pairs; its host blocks return to the host free
+ * list at the end of that step) instead of being recomputed. A victim that does
+ * not qualify, or finds too few host blocks, is recomputed as before.
+ * 0 turns swapping off. Call before the first step.
+ */
+pa_status pa_sched_set_swap(pa_sched* s, int32_t num_host_blocks);
 void pa_sched_destroy(pa_sched* s);
 
 #ifdef __cplusplus

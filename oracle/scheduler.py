@@ -32,6 +32,11 @@ Readings where the pages are silent or loose (listed in the design notes):
     hold that request);
   * prompt K/V is (re)written only for requests admitted this step that are
     still running at its end;
+  * swap mode: a victim whose KV was written before the step and whose
+    blocks are not shared is copied to host blocks (FIFO host free list)
+    instead of being dropped, and copied back into fresh blocks when admitted
+    again; its host blocks are free again after that step; victims that do
+    not qualify or find too few host blocks are recomputed;
   * with prompt token ids (prefix caching), admission allocates through the
     block manager's prefix cache and the prompt K/V is written from the first
     position not covered by already-written cached blocks; the blocks of
@@ -69,6 +74,18 @@ class OracleScheduler:
         self.n_finished = 0
         self.step_idx = 0
         self.tokens = None   # per-request prompt token ids when prefix caching is used
+        # swap-mode preemption ("vLLM 原理" / "Preemption（抢占）": Swap mode moves the
+        # KV cache to the CPU; "PagedAttention与Continuous Batching原理与实践" §3.4 --swap-space)
+        self.swap = False
+        self.host_free: deque[int] = deque()
+        self.host_table: dict[int, list[int]] = {}
+        self.swapping_in: set[int] = set()
+
+    def set_swap(self, num_host_blocks: int) -> None:
+        if self.step_idx != 0 or num_host_blocks < 0:
+            raise BMError("INVALID_ARG", "before the first step")
+        self.swap = num_host_blocks > 0
+        self.host_free = deque(range(num_host_blocks))
 
     def set_prompt_tokens(self, tokens) -> None:
         """Prompt token ids per request; admission then reuses cached prompt
@@ -102,8 +119,15 @@ class OracleScheduler:
         while self.waiting:
             r = self.waiting[0]
             total = self.prompt[r] + self.generated[r]
+            from_host = bool(self.host_table.get(r))
             try:
-                if self.tokens is None:
+                if from_host:
+                    # swapped out earlier: its KV is copied back, nothing recomputed
+                    if blocks_for(total) > bm.num_free():
+                        raise BMError("NO_BLOCKS", "")
+                    bm.allocate(r, total)
+                    start = total
+                elif self.tokens is None:
                     if blocks_for(total) > bm.num_free():
                         raise BMError("NO_BLOCKS", "")
                     bm.allocate(r, total)
@@ -121,11 +145,35 @@ class OracleScheduler:
             admitted.append(r)
             admit_len[r] = total
             admit_start[r] = start
+            if from_host:
+                self.swapping_in.add(r)
+            else:
+                self.swapping_in.discard(r)
 
         # 4. grow every running request by one slot, preempting from the tail
         decode_slot = {}
         cow = []
         preempted = []
+        swap_out, swapped_out = [], []
+
+        def swap_out_or_drop(v):
+            """Swap-mode victim: copy its blocks to host blocks when its KV was
+            written before this step and no block is shared; a request that
+            came from host blocks this step keeps its host copy."""
+            if v in self.swapping_in:
+                self.swapping_in.discard(v)
+                return
+            self.host_table.pop(v, None)
+            if not self.swap or v in admitted:
+                return
+            table = bm.table(v)
+            if len(table) > len(self.host_free) or any(bm.refcount[b] != 1 for b in table):
+                return
+            host = [self.host_free.popleft() for _ in table]
+            self.host_table[v] = host
+            swap_out.extend(zip(table, host))
+            swapped_out.append(v)
+
         i = 0
         stop = False
         while i < len(self.running) and not stop:
@@ -137,6 +185,7 @@ class OracleScheduler:
                     if e.status != "NO_BLOCKS":
                         raise
                     victim = self.running.pop()
+                    swap_out_or_drop(victim)
                     bm.free(victim)
                     self.waiting.appendleft(victim)
                     preempted.append(victim)
@@ -155,7 +204,15 @@ class OracleScheduler:
         # 5. the step's device work, described by index arrays
         running = list(self.running)
         still = set(running)
-        prompt_seqs = [r for r in admitted if r in still]
+        swap_in, swapped_in = [], []
+        for r in admitted:
+            if r in still and r in self.swapping_in:
+                host = self.host_table.pop(r)
+                swap_in.extend(zip(host, bm.table(r)))
+                self.host_free.extend(host)       # free once this step's copies are queued
+                self.swapping_in.discard(r)
+                swapped_in.append(r)
+        prompt_seqs = [r for r in admitted if r in still and r not in swapped_in]
         prompt_slots = []
         for r in prompt_seqs:
             prompt_slots.extend(bm.slots(r, admit_start[r], admit_len[r] - admit_start[r]))
@@ -189,4 +246,8 @@ class OracleScheduler:
             "finished": finished,
             "num_waiting": len(self.waiting),
             "num_free_blocks": bm.num_free(),
+            "swap_out": swap_out,
+            "swap_in": swap_in,
+            "swapped_out": swapped_out,
+            "swapped_in": swapped_in,
         }

@@ -56,6 +56,10 @@ class pa_step_out(C.Structure):
         ("num_finished", C.c_int32), ("finished", _P64),
         ("num_waiting", C.c_int32), ("num_free_blocks", C.c_int32),
         ("prompt_starts", _P32), ("num_cached_tokens", C.c_int32),
+        ("num_swap_out", C.c_int32), ("swap_out_src", _P32), ("swap_out_dst", _P32),
+        ("num_swap_in", C.c_int32), ("swap_in_src", _P32), ("swap_in_dst", _P32),
+        ("num_swapped_out", C.c_int32), ("swapped_out", _P64),
+        ("num_swapped_in", C.c_int32), ("swapped_in", _P64),
     ]
 
 
@@ -94,6 +98,8 @@ def _declare(lib):
         "pa_sched_step": (i32, [vp, C.POINTER(pa_step_out)]),
         "pa_sched_destroy": (None, [vp]),
         "pa_sched_set_prompt_tokens": (i32, [vp, _P32, _P64]),
+        "pa_sched_set_swap": (i32, [vp, i32]),
+        "pa_copy_blocks_between": (i32, [vp, i32, vp, i32, vp, vp, i32, pa_pool_desc, vp]),
         "pa_bm_set_prefix_caching": (i32, [vp, i32]),
         "pa_bm_allocate_prefix": (i32, [vp, i64, _P32, i32, i32, _P32]),
         "pa_bm_mark_written": (i32, [vp, i64]),
@@ -265,6 +271,29 @@ def pa_copy_blocks(kv_pool, src, dst, stream=None):
         n, desc, _stream(stream)))
 
 
+def pa_copy_blocks_between(dst_pool, src_pool, src, dst, stream=None):
+    """Block copy between two pools of one block shape (device or pinned host)."""
+    desc = pool_desc(dst_pool)
+    if pool_desc(src_pool).num_kv_heads != desc.num_kv_heads or src_pool.shape[1:] != dst_pool.shape[1:] \
+            or src_pool.dtype != dst_pool.dtype:
+        raise ValueError("pools differ in block shape")
+    n = src.numel()
+    if dst.numel() != n:
+        raise ValueError("src and dst differ in length")
+    if n == 0:
+        return
+    for t, name in ((dst_pool, "dst_pool"), (src_pool, "src_pool"), (src, "src"), (dst, "dst")):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if not (t.is_cuda or t.is_pinned()):
+            raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    if src.dtype != torch.int32 or dst.dtype != torch.int32:
+        raise ValueError("src and dst must be int32")
+    _check("pa_copy_blocks_between", lib().pa_copy_blocks_between(
+        C.c_void_p(dst_pool.data_ptr()), dst_pool.shape[0], C.c_void_p(src_pool.data_ptr()), src_pool.shape[0],
+        C.c_void_p(src.data_ptr()), C.c_void_p(dst.data_ptr()), n, desc, _stream(stream)))
+
+
 def pa_get_device_error(stream=None) -> int:
     """Synchronises the stream, returns and clears the device error bits."""
     flags = C.c_uint32(0)
@@ -431,6 +460,10 @@ class Scheduler:
         _check("pa_sched_set_prompt_tokens", lib().pa_sched_set_prompt_tokens(self.handle, _i32p(flat),
                                                                               _i64p(offs)))
 
+    def set_swap(self, num_host_blocks: int):
+        """Swap-mode preemption with this many host blocks (0: recompute only)."""
+        _check("pa_sched_set_swap", lib().pa_sched_set_swap(self.handle, int(num_host_blocks)))
+
     def step_raw(self) -> pa_step_out:
         """Runs one step; the returned struct's arrays are valid until the next."""
         _check("pa_sched_step", lib().pa_sched_step(self.handle, C.byref(self._out)))
@@ -464,6 +497,12 @@ class Scheduler:
             "num_waiting": o.num_waiting, "num_free_blocks": o.num_free_blocks,
             "prompt_starts": arr(o.prompt_starts, o.num_prompt_seqs, np.int32),
             "num_cached_tokens": o.num_cached_tokens,
+            "swap_out": list(zip(arr(o.swap_out_src, o.num_swap_out, np.int32).tolist(),
+                                 arr(o.swap_out_dst, o.num_swap_out, np.int32).tolist())),
+            "swap_in": list(zip(arr(o.swap_in_src, o.num_swap_in, np.int32).tolist(),
+                                arr(o.swap_in_dst, o.num_swap_in, np.int32).tolist())),
+            "swapped_out": arr(o.swapped_out, o.num_swapped_out, np.int64),
+            "swapped_in": arr(o.swapped_in, o.num_swapped_in, np.int64),
         }
 
 

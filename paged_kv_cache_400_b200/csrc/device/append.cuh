@@ -57,4 +57,27 @@ copy_blocks_kernel(uint4* __restrict__ pool, const int32_t* __restrict__ src,
   for (int64_t i = threadIdx.x; i < chunks_per_block; i += blockDim.x) to[i] = from[i];
 }
 
+// Whole-block copy between two pools of the same block shape (device <->
+// pinned host for swapping, or device <-> device): pair i copies block src[i]
+// of `from` to block dst[i] of `to`. Each block is split across `split` CTAs
+// so that even a few pairs keep many 16-byte transfers in flight (a PCIe or
+// C2C link needs that to reach its bandwidth).
+__global__ void __launch_bounds__(256)
+copy_blocks_between_kernel(uint4* __restrict__ to, int32_t to_blocks, const uint4* __restrict__ from,
+                           int32_t from_blocks, const int32_t* __restrict__ src, const int32_t* __restrict__ dst,
+                           int64_t chunks_per_block, int32_t split) {
+  const int32_t pair = blockIdx.x / split;
+  const int32_t part = blockIdx.x % split;
+  const int32_t s = src[pair];
+  const int32_t d = dst[pair];
+  if (s < 0 || s >= from_blocks || d < 0 || d >= to_blocks) {
+    if (threadIdx.x == 0 && part == 0) raise_device_error(PA_DEVERR_BLOCK);
+    return;
+  }
+  const int64_t per = chunks_per_block / split;
+  const uint4* a = from + (int64_t)s * chunks_per_block + part * per;
+  uint4* b = to + (int64_t)d * chunks_per_block + part * per;
+  for (int64_t i = threadIdx.x; i < per; i += blockDim.x) b[i] = a[i];
+}
+
 }  // namespace pagedkv

@@ -318,6 +318,61 @@ pa_status pa_copy_blocks(void* kv_pool, const int32_t* src, const int32_t* dst, 
   return launch_status("pa_copy_blocks");
 }
 
+namespace {
+
+// A pool the GPU can address: device memory, or pinned host memory mapped
+// into the device's address space (checked at both ends of the range).
+pa_status check_addressable(const void* p, size_t bytes, const char* fn, const char* name) {
+  for (const char* q : {static_cast<const char*>(p), static_cast<const char*>(p) + bytes - 1}) {
+    cudaPointerAttributes a;
+    cudaError_t e = cudaPointerGetAttributes(&a, q);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(PA_ERR_INVALID_ARG, "%s: %s is not memory the GPU can address (%s)", fn, name,
+                  cudaGetErrorString(e));
+    }
+    const bool ok = (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged ||
+                     (a.type == cudaMemoryTypeHost && a.devicePointer == q));
+    if (!ok)
+      return fail(PA_ERR_INVALID_ARG, "%s: %s must be device memory or mapped pinned host memory", fn, name);
+  }
+  return PA_OK;
+}
+
+}  // namespace
+
+pa_status pa_copy_blocks_between(void* dst_pool, int32_t dst_num_blocks, const void* src_pool,
+                                 int32_t src_num_blocks, const int32_t* src, const int32_t* dst, int32_t n,
+                                 pa_pool_desc pool, void* stream) {
+  pa_pool_desc d = pool;
+  d.num_blocks = 1;
+  pa_status s = check_pool(d, "pa_copy_blocks_between");
+  if (s != PA_OK) return s;
+  if (n < 0 || dst_num_blocks <= 0 || src_num_blocks <= 0)
+    return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks_between: n %d, blocks %d / %d", n, dst_num_blocks,
+                src_num_blocks);
+  if (n == 0) return PA_OK;
+  if (!dst_pool || !src_pool || !src || !dst)
+    return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks_between: NULL pointer");
+  if (!aligned16(dst_pool) || !aligned16(src_pool))
+    return fail(PA_ERR_INVALID_ARG, "pa_copy_blocks_between: pools must be 16-byte aligned");
+  const size_t block_bytes =
+      (size_t)2 * pool.num_kv_heads * PA_BLOCK_SIZE * pool.head_dim * elem_size(pool.dtype);
+  if ((s = check_addressable(dst_pool, block_bytes * dst_num_blocks, "pa_copy_blocks_between", "dst_pool")) != PA_OK)
+    return s;
+  if ((s = check_addressable(src_pool, block_bytes * src_num_blocks, "pa_copy_blocks_between", "src_pool")) != PA_OK)
+    return s;
+  if ((s = check_addressable(src, sizeof(int32_t) * n, "pa_copy_blocks_between", "src")) != PA_OK) return s;
+  if ((s = check_addressable(dst, sizeof(int32_t) * n, "pa_copy_blocks_between", "dst")) != PA_OK) return s;
+  const int64_t chunks = (int64_t)(block_bytes / 16);
+  int32_t split = 1;
+  while (split < 16 && (chunks % (split * 2)) == 0 && chunks / (split * 2) >= 256) split *= 2;
+  pagedkv::copy_blocks_between_kernel<<<(unsigned)(n * split), 256, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<uint4*>(dst_pool), dst_num_blocks, reinterpret_cast<const uint4*>(src_pool),
+      src_num_blocks, src, dst, chunks, split);
+  return launch_status("pa_copy_blocks_between");
+}
+
 pa_status pa_get_device_error(uint32_t* flags, void* stream) {
   if (!flags) return fail(PA_ERR_INVALID_ARG, "pa_get_device_error: flags is NULL");
   void* addr = nullptr;

@@ -37,6 +37,13 @@ struct pa_sched {
   std::vector<int32_t> admit_start;         // first position whose KV the admission writes
   std::vector<int32_t> tokens;              // prompt token ids (prefix caching), or empty
   std::vector<int64_t> token_offset;        // request i's prompt: tokens[token_offset[i] ...]
+  // swap-mode preemption: host blocks (FIFO free list) hold preempted KV
+  bool swap = false;
+  int32_t host_blocks = 0;
+  std::deque<int32_t> host_free;
+  std::vector<std::vector<int32_t>> host_table;  // per request: its KV in host blocks, or empty
+  std::vector<int32_t> swapped_len;              // tokens of KV held in host_table
+  std::vector<char> swapping_in;                 // admitted this step from host blocks
   int32_t n_finished = 0;
   int32_t step_idx = 0;
   // step outputs
@@ -44,6 +51,8 @@ struct pa_sched {
   std::vector<int64_t> o_admitted, o_preempted, o_finished;
   std::vector<int32_t> o_seq_lens, o_block_tables, o_prompt_lens, o_cow_src, o_cow_dst, o_prompt_starts;
   int32_t o_cached_tokens = 0;
+  std::vector<int32_t> o_swap_out_src, o_swap_out_dst, o_swap_in_src, o_swap_in_dst;
+  std::vector<int64_t> o_swapped_out, o_swapped_in;
   std::vector<int64_t> slot_of;  // per request: slot appended this step
 };
 
@@ -74,6 +83,51 @@ void publish(pa_sched* s, pa_step_out* out) {
   out->num_free_blocks = s->bm->free_blocks();
   out->prompt_starts = s->o_prompt_starts.data();
   out->num_cached_tokens = s->o_cached_tokens;
+  out->num_swap_out = (int32_t)s->o_swap_out_src.size();
+  out->swap_out_src = s->o_swap_out_src.data();
+  out->swap_out_dst = s->o_swap_out_dst.data();
+  out->num_swap_in = (int32_t)s->o_swap_in_src.size();
+  out->swap_in_src = s->o_swap_in_src.data();
+  out->swap_in_dst = s->o_swap_in_dst.data();
+  out->num_swapped_out = (int32_t)s->o_swapped_out.size();
+  out->swapped_out = s->o_swapped_out.data();
+  out->num_swapped_in = (int32_t)s->o_swapped_in.size();
+  out->swapped_in = s->o_swapped_in.data();
+}
+
+// Preemption victim v in swap mode: when its KV was written before this step
+// and none of its blocks is shared, its blocks are copied to host blocks
+// (swap-out pairs, run before any other device work of the step) and it will
+// come back by copying instead of recomputing. A request admitted from host
+// blocks in this same step keeps its host copy. Otherwise (no swap mode, not
+// enough host blocks, shared blocks, KV not yet written) it is recomputed.
+pa_status swap_out_or_drop(pa_sched* s, int64_t v) {
+  pa_bm* bm = s->bm;
+  if (s->swapping_in[v]) {  // its KV is still in host blocks
+    s->swapping_in[v] = 0;
+    return PA_OK;
+  }
+  s->host_table[v].clear();
+  if (!s->swap) return PA_OK;
+  bool admitted_now = false;
+  for (int64_t r : s->o_admitted) admitted_now |= (r == v);
+  if (admitted_now) return PA_OK;
+  auto it = bm->seqs.find(v);
+  if (it == bm->seqs.end()) return fail(PA_ERR_UNKNOWN_SEQ, "pa_sched_step: victim %lld", (long long)v);
+  const std::vector<int32_t>& table = it->second.table;
+  if ((int32_t)table.size() > (int32_t)s->host_free.size()) return PA_OK;
+  for (int32_t b : table)
+    if (bm->refcount[b] != 1) return PA_OK;
+  for (int32_t b : table) {
+    const int32_t h = s->host_free.front();
+    s->host_free.pop_front();
+    s->host_table[v].push_back(h);
+    s->o_swap_out_src.push_back(b);
+    s->o_swap_out_dst.push_back(h);
+  }
+  s->swapped_len[v] = it->second.len;
+  s->o_swapped_out.push_back(v);
+  return PA_OK;
 }
 
 }  // namespace
@@ -107,6 +161,9 @@ pa_status pa_sched_create(pa_bm* bm, const int32_t* arrival_step, const int32_t*
   s->is_running.assign(n_requests, 0);
   s->admit_len.assign(n_requests, 0);
   s->admit_start.assign(n_requests, 0);
+  s->host_table.assign(n_requests, {});
+  s->swapped_len.assign(n_requests, 0);
+  s->swapping_in.assign(n_requests, 0);
   s->slot_of.assign(n_requests, -1);
   s->arrival_order.resize(n_requests);
   std::iota(s->arrival_order.begin(), s->arrival_order.end(), 0);
@@ -117,6 +174,16 @@ pa_status pa_sched_create(pa_bm* bm, const int32_t* arrival_step, const int32_t*
 }
 
 void pa_sched_destroy(pa_sched* s) { delete s; }
+
+pa_status pa_sched_set_swap(pa_sched* s, int32_t num_host_blocks) {
+  if (!s || num_host_blocks < 0) return fail(PA_ERR_INVALID_ARG, "pa_sched_set_swap: bad argument");
+  if (s->step_idx != 0) return fail(PA_ERR_INVALID_ARG, "pa_sched_set_swap: only before the first step");
+  s->swap = num_host_blocks > 0;
+  s->host_blocks = num_host_blocks;
+  s->host_free.clear();
+  for (int32_t i = 0; i < num_host_blocks; ++i) s->host_free.push_back(i);
+  return PA_OK;
+}
 
 pa_status pa_sched_set_prompt_tokens(pa_sched* s, const int32_t* tokens, const int64_t* offsets) {
   if (!s || !tokens || !offsets) return fail(PA_ERR_INVALID_ARG, "pa_sched_set_prompt_tokens: NULL argument");
@@ -151,6 +218,12 @@ pa_status pa_sched_step(pa_sched* s, pa_step_out* out) {
   s->o_cow_dst.clear();
   s->o_prompt_starts.clear();
   s->o_cached_tokens = 0;
+  s->o_swap_out_src.clear();
+  s->o_swap_out_dst.clear();
+  s->o_swap_in_src.clear();
+  s->o_swap_in_dst.clear();
+  s->o_swapped_out.clear();
+  s->o_swapped_in.clear();
   out->step = step;
 
   // 1. retire requests that generated all their tokens; pages return at once
@@ -185,7 +258,12 @@ pa_status pa_sched_step(pa_sched* s, pa_step_out* out) {
     const int32_t total = s->prompt[r] + s->generated[r];
     int32_t cached = 0;
     pa_status st;
-    if (s->tokens.empty()) {
+    const bool from_host = !s->host_table[r].empty();
+    if (from_host) {
+      // swapped out earlier: fresh device blocks, KV copied back (no recompute)
+      st = pagedkv::blocks_for(total) > bm->free_blocks() ? PA_ERR_NO_BLOCKS : pa_bm_allocate(bm, r, total);
+      cached = total;
+    } else if (s->tokens.empty()) {
       st = pagedkv::blocks_for(total) > bm->free_blocks() ? PA_ERR_NO_BLOCKS : pa_bm_allocate(bm, r, total);
     } else {
       st = pa_bm_allocate_prefix(bm, r, s->tokens.data() + s->token_offset[r], s->prompt[r], total, &cached);
@@ -203,6 +281,7 @@ pa_status pa_sched_step(pa_sched* s, pa_step_out* out) {
     s->o_admitted.push_back(r);
     s->admit_len[r] = total;
     s->admit_start[r] = cached;
+    s->swapping_in[r] = from_host ? 1 : 0;
   }
 
   // 4. grow every running request by one slot; preempt the newest on shortage
@@ -224,6 +303,7 @@ pa_status pa_sched_step(pa_sched* s, pa_step_out* out) {
       if (st != PA_ERR_NO_BLOCKS) return st;
       const int64_t victim = s->running.back();
       s->running.pop_back();
+      if ((st = swap_out_or_drop(s, victim)) != PA_OK) return st;
       st = pa_bm_free(bm, victim);
       if (st != PA_OK) return st;
       s->is_running[victim] = 0;
@@ -253,6 +333,22 @@ pa_status pa_sched_step(pa_sched* s, pa_step_out* out) {
   for (size_t i = 0; i < nr; ++i) s->o_decode_slots[i] = s->slot_of[s->running[i]];
   for (int64_t r : s->o_admitted) {
     if (!s->is_running[r]) continue;  // admitted, then preempted in the same step
+    if (s->swapping_in[r]) {
+      // KV comes back from host blocks; those blocks are free after this step
+      auto it = bm->seqs.find(r);
+      if (it == bm->seqs.end()) return fail(PA_ERR_UNKNOWN_SEQ, "pa_sched_step: swapped-in %lld", (long long)r);
+      const std::vector<int32_t>& dev = it->second.table;  // may hold this step's new block too
+      const std::vector<int32_t>& host = s->host_table[r];
+      for (size_t i = 0; i < host.size(); ++i) {
+        s->o_swap_in_src.push_back(host[i]);
+        s->o_swap_in_dst.push_back(dev[i]);
+        s->host_free.push_back(host[i]);
+      }
+      s->host_table[r].clear();
+      s->swapping_in[r] = 0;
+      s->o_swapped_in.push_back(r);
+      continue;
+    }
     const int32_t n = s->admit_len[r];
     const int32_t start = s->admit_start[r];
     s->o_prompt_seqs.push_back(r);

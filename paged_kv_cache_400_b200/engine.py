@@ -50,6 +50,8 @@ class StepIndices:
     prompt_slots: np.ndarray
     cow_src: np.ndarray
     cow_dst: np.ndarray
+    swap_out: np.ndarray       # [n][2] (device block, host block)
+    swap_in: np.ndarray        # [n][2] (host block, device block)
     done: bool
     record: StepRecord = field(default=None)
 
@@ -57,10 +59,11 @@ class StepIndices:
 class DecodeEngine:
     def __init__(self, num_blocks, num_layers, num_heads, num_kv_heads, head_dim, arrival_step,
                  prompt_len, output_len, table_width, scale, device, dtype=torch.bfloat16,
-                 max_seq_len=None, prompt_tokens=None):
+                 max_seq_len=None, prompt_tokens=None, swap_host_blocks=0):
         """prompt_tokens: per-request prompt token ids to turn on automatic
         prefix caching (admission reuses cached prompt blocks and only the KV
-        after the cached prefix is written)."""
+        after the cached prefix is written). swap_host_blocks: pinned host
+        blocks per layer for swap-mode preemption (0: recompute only)."""
         self.device = torch.device(device)
         self.num_layers = num_layers
         self.num_heads = num_heads
@@ -75,8 +78,14 @@ class DecodeEngine:
         self.sched = bd.Scheduler(self.bm, arrival_step, prompt_len, output_len, table_width)
         if prompt_tokens is not None:
             self.sched.set_prompt_tokens(prompt_tokens)
+        self.host_pools = []
+        if swap_host_blocks > 0:
+            self.sched.set_swap(swap_host_blocks)
         shape = (num_blocks, 2, num_kv_heads, bd.BLOCK_SIZE, head_dim)
         self.pools = [torch.empty(shape, dtype=dtype, device=self.device) for _ in range(num_layers)]
+        if swap_host_blocks > 0:
+            hshape = (swap_host_blocks,) + shape[1:]
+            self.host_pools = [torch.empty(hshape, dtype=dtype, pin_memory=True) for _ in range(num_layers)]
         self._ws = None
         self._ws_bytes = 0
 
@@ -110,6 +119,10 @@ class DecodeEngine:
             prompt_slots=arr(o.prompt_slots, o.num_prompt_tokens, np.int64),
             cow_src=arr(o.cow_src, o.num_cow, np.int32),
             cow_dst=arr(o.cow_dst, o.num_cow, np.int32),
+            swap_out=np.stack([arr(o.swap_out_src, o.num_swap_out, np.int32),
+                               arr(o.swap_out_dst, o.num_swap_out, np.int32)], axis=1),
+            swap_in=np.stack([arr(o.swap_in_src, o.num_swap_in, np.int32),
+                              arr(o.swap_in_dst, o.num_swap_in, np.int32)], axis=1),
             done=bool(o.done),
         )
         idx.record = StepRecord(o.step, n, o.num_prompt_tokens, o.num_admitted, o.num_preempted,
@@ -139,6 +152,24 @@ class DecodeEngine:
             self._ws_bytes = need
         return self._ws
 
+    def run_swaps(self, idx: StepIndices):
+        """This step's swap copies, every layer: swap-out (device -> host) before
+        swap-in (host -> device), both before any other write of the step."""
+        if not len(idx.swap_out) and not len(idx.swap_in):
+            return
+        dev = self.device
+        pairs = [(idx.swap_out, False), (idx.swap_in, True)]
+        for arr, to_device in pairs:
+            if not len(arr):
+                continue
+            src = torch.from_numpy(np.ascontiguousarray(arr[:, 0])).to(dev)
+            dst = torch.from_numpy(np.ascontiguousarray(arr[:, 1])).to(dev)
+            for pool, host in zip(self.pools, self.host_pools):
+                if to_device:
+                    bd.pa_copy_blocks_between(pool, host, src, dst)
+                else:
+                    bd.pa_copy_blocks_between(host, pool, src, dst)
+
     def run_layers(self, idx: StepIndices, inputs, out=None):
         """Device work of one step over all layers.
 
@@ -157,6 +188,7 @@ class DecodeEngine:
         cs = torch.from_numpy(idx.cow_src).to(dev) if len(idx.cow_src) else None
         cd = torch.from_numpy(idx.cow_dst).to(dev) if len(idx.cow_dst) else None
         ws = self.workspace(n)
+        self.run_swaps(idx)
         outs = out if out is not None else [torch.empty(n, self.num_heads, self.head_dim,
                                                          dtype=self.pools[0].dtype, device=dev)
                                              for _ in range(self.num_layers)]
@@ -240,6 +272,7 @@ class GraphedLayers:
         nb = ((n + self.bucket - 1) // self.bucket) * self.bucket
         graph = self._graph(nb)  # captured on first use, before the rows are filled
         # eager, variable-size work first
+        e.run_swaps(idx)
         cs = torch.from_numpy(idx.cow_src).to(dev) if len(idx.cow_src) else None
         cd = torch.from_numpy(idx.cow_dst).to(dev) if len(idx.cow_dst) else None
         ps = torch.from_numpy(idx.prompt_slots).to(dev, non_blocking=True) if len(idx.prompt_slots) else None

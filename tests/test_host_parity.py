@@ -145,3 +145,30 @@ def test_scheduler_rejects_oversized_request():
     with pytest.raises(bd.PagedKVError) as e:
         bd.Scheduler(bm, [0], [100], [100], 4)
     assert e.value.status == "CAPACITY"
+
+
+@pytest.mark.parametrize("host_blocks", [0, 300, 5000])
+def test_swap_mode_trace_replay_is_identical(host_blocks):
+    """Swap-mode preemption (few host blocks: swap and recompute mixed; many:
+    every eligible victim swapped) replays identically in C++ and the oracle."""
+    case = wl.trace_case(seed=3, n_requests=300, rate=20.0, num_blocks=2500, num_layers=1)
+    obm, cbm = OracleBlockManager(case.num_blocks), bd.BlockManager(case.num_blocks)
+    osch = OracleScheduler(obm, case.arrival_step, case.prompt_len, case.output_len, case.table_width)
+    csch = bd.Scheduler(cbm, case.arrival_step, case.prompt_len, case.output_len, case.table_width)
+    osch.set_swap(host_blocks)
+    csch.set_swap(host_blocks)
+    outs = swapped = 0
+    while True:
+        o, c = osch.step(), csch.step()
+        compare_steps(o, c)
+        assert o["swap_out"] == c["swap_out"] and o["swap_in"] == c["swap_in"]
+        assert list(o["swapped_out"]) == c["swapped_out"].tolist()
+        assert list(o["swapped_in"]) == c["swapped_in"].tolist()
+        outs += len(o["preempted"])
+        swapped += len(o["swapped_out"])
+        if o["done"]:
+            break
+    assert outs > 0
+    assert (swapped > 0) == (host_blocks > 0)
+    if host_blocks == 300:
+        assert 0 < swapped < outs
