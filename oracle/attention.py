@@ -189,3 +189,35 @@ def copy_blocks(pool, src, dst):
             continue
         pool[d] = pool[s]
     return rejected
+
+
+# --------------------------------------------------------------------------
+# prefill / chunked prefill: the new tokens of each sequence attend causally
+# --------------------------------------------------------------------------
+def paged_prefill(q, pool, block_tables, seq_lens, query_lens, scale: float, dtype: str):
+    """Causal attention of each sequence's newest query_lens[b] tokens.
+
+    Sequence b holds seq_lens[b] tokens of KV (its new tokens included, as the
+    last query_lens[b] positions). Query row i of sequence b (rows of q are the
+    sequences' new tokens, concatenated in order) sits at position
+    p = seq_lens[b] - query_lens[b] + i and attends to positions 0..p
+    ("PagedAttention与Continuous Batching原理与实践" §2: prefill processes the
+    whole prompt; each token sees itself and every earlier token).
+    q: [sum(query_lens)][H][D] in storage dtype; returns fp64 of that shape."""
+    qf = to_f64(q, dtype)
+    T, H, D = qf.shape
+    G = H // pool.shape[2]
+    out = np.zeros((T, H, D), dtype=np.float64)
+    row = 0
+    for b, (L, n) in enumerate(zip(seq_lens, query_lens)):
+        L, n = int(L), int(n)
+        if n == 0:
+            continue
+        K, V = gather_kv(pool, block_tables[b], L, dtype)
+        for i in range(n):
+            p = L - n + i
+            for h in range(H):
+                g = h // G
+                out[row + i, h] = softmax_attention(qf[row + i, h], K[:p + 1, g, :], V[:p + 1, g, :], scale)
+        row += n
+    return out

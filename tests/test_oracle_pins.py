@@ -375,3 +375,41 @@ def test_copy_blocks_bits_and_bounds():
     assert rejected == [2]
     assert np.array_equal(pool[4], orig[1]) and np.array_equal(pool[0], orig[3])
     assert np.array_equal(pool[[1, 2, 3]], orig[[1, 2, 3]])
+
+
+# ---------------------------------------------------------------------------
+# prefill (causal) oracle
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("n_heads,n_kv", [(4, 4), (8, 2)])
+def test_prefill_matches_causal_sdpa(n_heads, n_kv):
+    rng = np.random.default_rng(20 + n_heads)
+    lens, qlens = [1, 17, 40, 70], [1, 17, 12, 33]     # full prompts and chunks after a context
+    d = 16
+    K, V = random_logical(rng, lens, n_kv, d)
+    pool, tables = scatter_logical(K, V, 32, rng)
+    q = rng.standard_normal((sum(qlens), n_heads, d))
+    out = oa.paged_prefill(q, pool, tables, lens, qlens, 0.3, "f64")
+    G = n_heads // n_kv
+    row = 0
+    for b, (L, n) in enumerate(zip(lens, qlens)):
+        kt = torch.from_numpy(K[b]).permute(1, 0, 2).repeat_interleave(G, dim=0)[None]
+        vt = torch.from_numpy(V[b]).permute(1, 0, 2).repeat_interleave(G, dim=0)[None]
+        qt = torch.from_numpy(q[row:row + n]).permute(1, 0, 2)[None]
+        # causal with the queries at the last n positions: mask[i, t] = t <= L - n + i
+        mask = torch.arange(L)[None, :] <= (L - n + torch.arange(n))[:, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=0.3)
+        np.testing.assert_allclose(out[row:row + n], ref[0].permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+        row += n
+
+
+def test_prefill_last_row_is_decode_and_first_token_sees_itself():
+    rng = np.random.default_rng(30)
+    lens, qlens = [33], [33]
+    K, V = random_logical(rng, lens, 2, 8)
+    pool, tables = scatter_logical(K, V, 8, rng)
+    q = rng.standard_normal((33, 4, 8))
+    pre = oa.paged_prefill(q, pool, tables, lens, qlens, 0.5, "f64")
+    dec = oa.paged_decode(q[-1:], pool, tables, lens, 0.5, "f64")
+    assert np.array_equal(pre[-1], dec[0])
+    for h in range(4):
+        assert np.array_equal(pre[0, h], V[0][0, h // 2])
