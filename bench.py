@@ -47,7 +47,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--workload", choices=["gqa", "mha", "prefix", "trace", "prefix_trace"], default="gqa",
+    ap.add_argument("--workload", choices=["gqa", "mha", "prefix", "trace", "prefix_trace", "prefill",
+                                           "chunked_prefill"], default="gqa",
                     help="gqa is the benchmark line; the others are extra measurements")
     ap.add_argument("--trace-layers", type=int, default=32)
     ap.add_argument("--trace-requests", type=int, default=2000)
@@ -578,6 +579,166 @@ def run_trace(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def prefill_flops(case):
+    """Algorithmic FLOPs of causal prefill attention: a new token at position p
+    scores p + 1 keys and sums p + 1 values, 2 x 128 FLOPs each, per query head."""
+    f = 0
+    for c, n in zip(case.ctx_lens, case.query_lens):
+        # sum over p = c .. c+n-1 of (p + 1)
+        f += n * c + n * (n + 1) // 2
+    return 4 * case.head_dim * case.num_heads * f
+
+
+def measured_tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    except Exception:
+        return 1590.0, "fallback 1.59 PFLOP/s"
+
+
+def oracle_prefill_sample(case, seconds, rng_seed=0):
+    """The oracle (as it stands) on whole sequences of the step in random
+    order, for about `seconds`: append of the new tokens' K/V, then causal fp64
+    attention. Input generation is outside the timed part. Returns (new tokens
+    done, sequences done, oracle seconds)."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from oracle_side import oracle_prefill_compute, oracle_prefill_indices, oracle_prefill_inputs
+    ost = oracle_prefill_indices(case)
+    order = np.random.default_rng(rng_seed).permutation(len(case.query_lens))
+    toks = done = 0
+    busy = 0.0
+    while done < len(order) and busy < seconds:
+        b = int(order[done])
+        x = oracle_prefill_inputs(case, ost, [b])
+        t0 = time.perf_counter()
+        oracle_prefill_compute(x)
+        busy += time.perf_counter() - t0
+        toks += case.query_lens[b]
+        done += 1
+    return toks, done, busy
+
+
+def run_prefill(args, rank, world, dist):
+    """One prefill step per iteration: append every new token's K/V into its
+    slot (pa_reshape_and_cache), then causal paged attention of the new tokens
+    (pa_prefill). Reports new tokens per second and the attention kernel's
+    TFLOP/s against the measured bf16 tensor peak."""
+    import torch
+
+    import paged_kv_cache_400_b200 as pk
+    from paged_kv_cache_400_b200 import workloads as wl
+    from paged_kv_cache_400_b200.scenario import prepare_prefill_step
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    chunked = args.workload == "chunked_prefill"
+    case = (wl.chunked_prefill_case(args.seed + rank) if chunked else wl.prefill_case(args.seed + rank))
+    prep = prepare_prefill_step(case)
+    T = case.num_tokens
+    pool = case.make_pool(dev)
+    q = case.make_q(dev)
+    k, v = case.make_kv_new(dev)
+    slots = torch.from_numpy(prep.slot_mapping).to(dev)
+    bt = torch.from_numpy(prep.block_tables).to(dev)
+    sl = torch.from_numpy(prep.seq_lens).to(dev)
+    qs = torch.from_numpy(prep.query_start).to(dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    mq = case.max_query_len
+
+    def append():
+        pk.pa_reshape_and_cache(k, v, pool, slots)
+
+    def attend():
+        pk.pa_prefill(out, q, pool, bt, sl, qs, case.scale, mq)
+
+    for _ in range(max(args.warmup, 3)):
+        append()
+        attend()
+    assert pk.pa_get_device_error() == 0
+    K = args.steps
+    sampler = ClockSampler(local)
+    sampler.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    total_ms, (app_ms, att_ms) = timed_loop(K, stream, [append, attend])
+    wall1 = time.perf_counter()
+    if dist is not None:
+        dist.barrier()
+    sampler.stop()
+    assert pk.pa_get_device_error() == 0
+    total_ms = max_over_ranks(total_ms, dist, dev)
+    ms_per_step = total_ms / K
+    value = world * T / (ms_per_step / 1e3)
+
+    E = args.e2e_steps or min(K, 50)
+    pin = lambda t: t.cpu().pin_memory()
+    hs = [pin(t) for t in (q, k, v, slots, bt, sl, qs)]
+    h_out = torch.empty_like(out, device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in hs)
+    d2h = h_out.numel() * h_out.element_size()
+    for i in range(3 + E):
+        if i == 3:
+            if dist is not None:
+                dist.barrier()
+            torch.cuda.synchronize()
+            e0 = time.perf_counter()
+        for d_, h_ in zip((q, k, v, slots, bt, sl, qs), hs):
+            d_.copy_(h_, non_blocking=True)
+        append()
+        attend()
+        h_out.copy_(out, non_blocking=True)
+        stream.synchronize()
+    e2e_s = max_over_ranks((time.perf_counter() - e0) / E, dist, dev)
+    if rank != 0:
+        return
+    flops = prefill_flops(case)
+    att_avg = sum(att_ms) / K
+    peak, peak_src = measured_tensor_peak()
+    achieved = flops / (att_avg / 1e3) / 1e12
+    kv_bytes = int(sum(int(c) + int(n) for c, n in zip(case.ctx_lens, case.query_lens))) * 2 * \
+        case.num_kv_heads * case.head_dim * 2
+    desc = ("chunked_prefill_gqa: 64 sequences, cached context U[0,3072] + a 512-token chunk"
+            if chunked else "prefill_gqa: 64 whole prompts, lengths U[16,1024]")
+    line = {
+        "metric": "paged prefill new tokens/s (append + causal paged attention)", "value": value,
+        "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": desc + "; 32 q / 8 kv heads, head_dim 128, bf16, block_size 16, random "
+                                      "placement; step = pa_reshape_and_cache + pa_prefill",
+                   "global_batch": len(case.query_lens) * world, "new_tokens": T,
+                   "max_query_len": mq, "kv_tokens": int(prep.seq_lens.sum()),
+                   "parallelism": f"dp{world} independent replicas (no exchange step)",
+                   "l2": "no flush: K/V read %.2f GB per step (> 126 MB L2), q/out %.2f GB"
+                         % (kv_bytes / 1e9, 2 * T * case.num_heads * case.head_dim * 2 / 1e9)},
+        "roofline": {"kernel": "prefill_kernel (pa_prefill)", "bound": "tensor", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_src,
+                     "traffic": None, "traffic_source": "not captured on this source",
+                     "algorithmic_flops_per_launch": flops, "avg_launch_ms": att_avg,
+                     "note": "mma.sync m16n8k16 (legacy tensor path on sm_100a)"},
+        "append_avg_ms": sum(app_ms) / K,
+        "gpu_launches": 2 * K,
+        "clocks": sampler.summary(wall0, wall1),
+        "e2e": {"value": world * T / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "note": "per step: H2D of q/k/v/slots/tables/lens/query_start from pinned memory, "
+                        "append, prefill, D2H of out, stream sync"},
+        "library": os.path.relpath(pk.library_path(), ROOT),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        toks, done, el = oracle_prefill_sample(case, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": toks / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{done} of {len(case.query_lens)} sequences ({toks} new tokens, random order): oracle "
+                      f"append + fp64 causal attention through its own block tables, {el:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -598,6 +759,8 @@ def main():
             run_reference(args, rank, world)
         elif args.workload in ("trace", "prefix_trace"):
             run_trace(args, rank, world)
+        elif args.workload in ("prefill", "chunked_prefill"):
+            run_prefill(args, rank, world, dist)
         else:
             run_ours(args, rank, world, dist)
     finally:

@@ -217,6 +217,39 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* kv_pool,
                             void* stream);
 
 /*
+ * Paged prefill / chunked-prefill attention: causal attention of each
+ * sequence's new tokens over its paged KV ([A] §2: prefill processes the whole
+ * prompt at once; [A] §2.2 / [B] "工作原理": KV is read through the page table).
+ * Sequence b holds seq_lens[b] tokens of KV, its n_b = query_start[b+1] -
+ * query_start[b] new tokens included as the last n_b positions (their K/V
+ * already appended, e.g. by pa_reshape_and_cache with the prompt's slots).
+ * Query row query_start[b] + i sits at position p = seq_lens[b] - n_b + i and
+ * attends to positions 0..p:
+ *     out[r, h, :] = sum_{t<=p} softmax_t(scale * q[r, h, :] . K_t[h / G]) V_t[h / G]
+ * A whole prompt is n_b = seq_lens[b]; a later chunk has n_b < seq_lens[b].
+ *   out, q: device [num_tokens][num_heads][head_dim] bf16, 16-byte aligned,
+ *       row-major; out is written only at the new tokens' rows.
+ *   block_tables: device int32 [num_seqs][max_blocks_per_seq];
+ *   seq_lens: device int32 [num_seqs]; query_start: device int32 [num_seqs+1]
+ *       (normally query_start[0] = 0, non-decreasing, query_start[num_seqs] =
+ *       num_tokens).
+ *   max_query_len: host bound on n_b (sizes the grid), <= num_tokens; 0
+ *       launches nothing.
+ * Supported: bf16 pools with head_dim 128, num_heads / num_kv_heads in
+ * {1, 2, 4, 8, 16} (else PA_ERR_UNSUPPORTED). Device-side checks: n_b < 0,
+ * n_b > max_query_len, query_start[b] < 0, query_start[b+1] > num_tokens,
+ * n_b > seq_lens[b] or seq_lens[b] > 16 * max_blocks_per_seq sets
+ * PA_DEVERR_SEQLEN and skips sequence b; a block id outside the pool sets
+ * PA_DEVERR_BLOCK (that block's contribution is undefined, nothing is read
+ * from it). Allocates nothing.
+ */
+pa_status pa_prefill(void* out, const void* q, const void* kv_pool,
+                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                     const int32_t* seq_lens, const int32_t* query_start,
+                     int32_t num_seqs, int32_t num_tokens, int32_t num_heads, float scale,
+                     pa_pool_desc pool, int32_t max_query_len, void* stream);
+
+/*
  * Block copy for copy-on-write: for i in [0, n) in order,
  *     kv_pool[dst[i]] = kv_pool[src[i]]    (the whole block: K and V, all heads).
  * src, dst: device int32 [n]. Pairs must not overlap (no block is both a source

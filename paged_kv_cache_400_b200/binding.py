@@ -105,6 +105,7 @@ def _declare(lib):
         "pa_bm_mark_written": (i32, [vp, i64]),
         "pa_bm_evictable_list": (i32, [vp, _P32, i32, _P32]),
         "pa_bm_num_cached": (i32, [vp]),
+        "pa_prefill": (i32, [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, f32, pa_pool_desc, i32, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -234,6 +235,25 @@ def pa_append_decode(out, q, k_new, v_new, kv_pool, slot_mapping, block_tables, 
         _dev(slot_mapping, "slot_mapping", torch.int64), _dev(block_tables, "block_tables", torch.int32),
         block_tables.shape[1], _dev(seq_lens, "seq_lens", torch.int32), B, H, float(scale), desc, ws_ptr,
         ws_bytes, int(max_seq_len), _stream(stream)))
+
+
+def pa_prefill(out, q, kv_pool, block_tables, seq_lens, query_start, scale, max_query_len, stream=None):
+    """Causal attention of each sequence's new tokens (the last
+    query_start[b+1] - query_start[b] positions of seq_lens[b]) over its paged
+    KV; q, out: [total new tokens][num_heads][128] bf16."""
+    desc = pool_desc(kv_pool)
+    T, H, D = q.shape
+    B = seq_lens.shape[0]
+    if out.shape != q.shape or D != desc.head_dim:
+        raise ValueError("q, out must be [num_tokens][num_heads][head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.shape != (B,) \
+            or query_start.shape != (B + 1,):
+        raise ValueError("block_tables [num_seqs][max_blocks], seq_lens [num_seqs], query_start [num_seqs+1]")
+    _check("pa_prefill", lib().pa_prefill(
+        _dev(out, "out", kv_pool.dtype), _dev(q, "q", kv_pool.dtype), _dev(kv_pool, "kv_pool"),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(seq_lens, "seq_lens", torch.int32), _dev(query_start, "query_start", torch.int32), B, T, H,
+        float(scale), desc, int(max_query_len), _stream(stream)))
 
 
 def pa_decode_noalloc(out, q, kv_pool, block_tables, seq_lens, scale, max_seq_len, stream=None):

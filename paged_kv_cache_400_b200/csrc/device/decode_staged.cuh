@@ -547,18 +547,18 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // Tensor map of a bf16 head_dim-128 pool: (d 128, row 16, kv head, K|V, block),
 // box (64, 16, 1, 2, 1), 128-byte swizzle, zero fill outside the tensor.
-inline pa_status encode_pool_map(const DecodeParams& p, CUtensorMap* map) {
+inline pa_status encode_pool_map(const void* pool, int32_t num_kv_heads, int32_t num_blocks, CUtensorMap* map) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) return fail(PA_ERR_CUDA, "pa_decode: cuTensorMapEncodeTiled unavailable");
-  const cuuint64_t hkv = (cuuint64_t)p.num_kv_heads;
-  const cuuint64_t dims[5] = {128, 16, hkv, 2, (cuuint64_t)p.num_blocks};
+  if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t hkv = (cuuint64_t)num_kv_heads;
+  const cuuint64_t dims[5] = {128, 16, hkv, 2, (cuuint64_t)num_blocks};
   const cuuint64_t strides[4] = {256, 4096, hkv * 4096, 2 * hkv * 4096};
   const cuuint32_t box[5] = {64, 16, 1, 2, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(p.pool), dims, strides, box,
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(pool), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "pa_decode: cuTensorMapEncodeTiled failed (%d)", (int)r);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return PA_OK;
 }
 
@@ -603,7 +603,7 @@ inline pa_status launch_staged_variant(const CUtensorMap& map, const DecodeParam
 
 inline pa_status launch_staged_bf16_d128(const DecodeParams& p, cudaStream_t st) {
   CUtensorMap map;
-  pa_status s = encode_pool_map(p, &map);
+  pa_status s = encode_pool_map(p.pool, p.num_kv_heads, p.num_blocks, &map);
   if (s != PA_OK) return s;
   if (p.work_items != nullptr) {
     decode_plan_kernel<<<1, kPlanThreads, 0, st>>>(p);

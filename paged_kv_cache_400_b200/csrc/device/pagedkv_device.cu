@@ -11,6 +11,7 @@
 #include "decode_common.cuh"
 #include "decode_generic.cuh"
 #include "decode_staged.cuh"
+#include "prefill.cuh"
 
 using pagedkv::fail;
 
@@ -301,6 +302,55 @@ pa_status pa_append_decode(void* out, const void* q, const void* k_new, const vo
   p.max_partitions = w.partitions > 0 ? w.partitions : 1;
   p.scale_log2 = scale * pagedkv::kLog2e;
   return pagedkv::launch_staged_bf16_d128(p, (cudaStream_t)stream);
+}
+
+pa_status pa_prefill(void* out, const void* q, const void* kv_pool, const int32_t* block_tables,
+                     int32_t max_blocks_per_seq, const int32_t* seq_lens, const int32_t* query_start,
+                     int32_t num_seqs, int32_t num_tokens, int32_t num_heads, float scale, pa_pool_desc pool,
+                     int32_t max_query_len, void* stream) {
+  pa_status s = check_pool(pool, "pa_prefill");
+  if (s != PA_OK) return s;
+  if (pool.dtype != PA_BF16 || pool.head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "pa_prefill: only bf16 pools with head_dim 128");
+  if (num_seqs < 0 || num_tokens < 0 || num_heads <= 0 || max_blocks_per_seq <= 0 || max_query_len < 0)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_prefill: num_seqs %d, num_tokens %d, num_heads %d, max_blocks %d, max_query_len %d", num_seqs,
+                num_tokens, num_heads, max_blocks_per_seq, max_query_len);
+  if (max_query_len > num_tokens)
+    return fail(PA_ERR_INVALID_ARG, "pa_prefill: max_query_len %d > num_tokens %d", max_query_len, num_tokens);
+  if (num_heads % pool.num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "pa_prefill: num_heads %d not a multiple of num_kv_heads %d", num_heads,
+                pool.num_kv_heads);
+  const int32_t G = num_heads / pool.num_kv_heads;
+  if (G > 16 || (G & (G - 1)) != 0)
+    return fail(PA_ERR_UNSUPPORTED, "pa_prefill: head group %d (1, 2, 4, 8 or 16)", G);
+  if (num_seqs > 65535 || pool.num_kv_heads > 65535)
+    return fail(PA_ERR_UNSUPPORTED, "pa_prefill: num_seqs %d or num_kv_heads %d > 65535", num_seqs,
+                pool.num_kv_heads);
+  if ((int64_t)max_query_len > (int64_t)max_blocks_per_seq * PA_BLOCK_SIZE)
+    return fail(PA_ERR_INVALID_ARG, "pa_prefill: max_query_len %d > max_blocks_per_seq * 16", max_query_len);
+  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "pa_prefill: scale is not finite");
+  if (num_seqs == 0 || max_query_len == 0) return PA_OK;
+  if (!out || !q || !kv_pool || !block_tables || !seq_lens || !query_start)
+    return fail(PA_ERR_INVALID_ARG, "pa_prefill: NULL pointer");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(kv_pool))
+    return fail(PA_ERR_INVALID_ARG, "pa_prefill: out, q and kv_pool must be 16-byte aligned");
+  pagedkv::PrefillParams p;
+  p.out = out;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.query_start = query_start;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_heads = num_heads;
+  p.num_kv_heads = pool.num_kv_heads;
+  p.group = G;
+  p.num_blocks = pool.num_blocks;
+  p.tile_tokens = 64 / G;
+  p.max_query_len = max_query_len;
+  p.num_tokens = num_tokens;
+  p.scale_log2 = scale * pagedkv::kLog2e;
+  return pagedkv::launch_prefill_bf16_d128(kv_pool, pool.num_blocks, p, num_seqs, (cudaStream_t)stream);
 }
 
 pa_status pa_copy_blocks(void* kv_pool, const int32_t* src, const int32_t* dst, int32_t n,

@@ -52,3 +52,26 @@ def prepare_decode_step(case) -> PreparedStep:
     bt, sl, _ = bm.pack(case.batch, case.table_width)
     return PreparedStep(bm, np.asarray(slots, np.int64), np.asarray(cs, np.int32),
                         np.asarray(cd, np.int32), bt, sl)
+
+
+@dataclass
+class PreparedPrefill:
+    bm: BlockManager
+    slot_mapping: np.ndarray     # int64 [T]: slot of each new token (sequence order)
+    block_tables: np.ndarray     # int32 [B][table_width]
+    seq_lens: np.ndarray         # int32 [B]: KV length, new tokens included
+    query_start: np.ndarray      # int32 [B+1]: first new-token row of each sequence
+
+
+def prepare_prefill_step(case) -> PreparedPrefill:
+    """Allocates every sequence's full length, then takes the slots of its new
+    positions ctx .. ctx+n-1 and packs the tables (all through the C ABI)."""
+    bm = BlockManager(case.num_blocks, case.free_order)
+    replay_ops(bm, case.ops)
+    seqs = list(range(len(case.query_lens)))
+    slots = [bm.slots(b, int(c), int(n)) for b, (c, n) in enumerate(zip(case.ctx_lens, case.query_lens))]
+    slot_mapping = np.concatenate(slots).astype(np.int64) if slots else np.zeros(0, np.int64)
+    bt, sl, _ = bm.pack(seqs, case.table_width)
+    qs = np.zeros(len(seqs) + 1, np.int32)
+    qs[1:] = np.cumsum(np.asarray(case.query_lens, np.int64))
+    return PreparedPrefill(bm, slot_mapping, bt, sl, qs)

@@ -30,6 +30,10 @@ Workloads (sizes follow the decode configurations they are named after):
   trace     2000 requests, Poisson(50) arrivals per step, prompts uniform in
             [16, 1024], outputs geometric with mean 200 capped at 2048,
             40000-block pool, 32/8 heads, head_dim 128, bf16.
+  prefill   64 whole prompts, lengths uniform in [16, 1024]; 32/8 heads,
+            head_dim 128, bf16, 16384-block pool.
+  chunked   64 sequences, cached context uniform in [0, 3072] plus a
+            512-token chunk; 32/8 heads, head_dim 128, bf16, 32768 blocks.
 Physical placement is random: the block manager's initial free list is a
 seeded permutation of the pool.
 """
@@ -267,6 +271,100 @@ def prefix_case(seed: int = 0) -> DecodeCase:
                       table_width=136, max_seq_len=2176,
                       info={"prefix_len": 1536, "suffix_lens": [int(x) for x in suffix],
                             "prompt_lens": plens, "samples": 4})
+
+
+# ---------------------------------------------------------------------------
+# prefill / chunked-prefill workloads
+# ---------------------------------------------------------------------------
+@dataclass
+class PrefillCase:
+    """One prefill step: sequence b holds ctx_lens[b] tokens of cached KV (from
+    the initial pool) and brings query_lens[b] new tokens, whose K/V
+    (k_new/v_new rows, in sequence order) are appended first; each new token
+    then attends causally over its sequence. The block manager allocates every
+    sequence's full length (ops) before the step."""
+    name: str
+    seed: int
+    num_blocks: int
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    dtype: str
+    scale: float
+    free_order: np.ndarray
+    ctx_lens: list
+    query_lens: list
+    table_width: int
+    info: dict = field(default_factory=dict)
+
+    pool_shape = DecodeCase.pool_shape
+    make_pool = DecodeCase.make_pool
+    pool_blocks = DecodeCase.pool_blocks
+
+    @property
+    def ops(self):
+        return [("allocate", b, int(c) + int(n))
+                for b, (c, n) in enumerate(zip(self.ctx_lens, self.query_lens))]
+
+    @property
+    def num_tokens(self) -> int:
+        return int(sum(self.query_lens))
+
+    @property
+    def max_query_len(self) -> int:
+        return int(max(self.query_lens)) if len(self.query_lens) else 0
+
+    def make_q(self, device="cpu") -> torch.Tensor:
+        return value_block(stream_key(self.seed, TAG_Q), (self.num_tokens, self.num_heads, self.head_dim),
+                           device=device, dtype=TORCH_DTYPE[self.dtype])
+
+    def make_kv_new(self, device="cpu"):
+        shape = (self.num_tokens, self.num_kv_heads, self.head_dim)
+        k = value_block(stream_key(self.seed, TAG_K), shape, device=device, dtype=TORCH_DTYPE[self.dtype])
+        v = value_block(stream_key(self.seed, TAG_V), shape, device=device, dtype=TORCH_DTYPE[self.dtype])
+        return k, v
+
+
+def prefill_custom(name, seed, ctx_lens, query_lens, num_heads=32, num_kv_heads=8,
+                   num_blocks=None, table_width=None) -> PrefillCase:
+    """A prefill step with caller-chosen lengths (bf16, head_dim 128)."""
+    rng = np.random.default_rng(seed + 707)
+    totals = [int(c) + int(n) for c, n in zip(ctx_lens, query_lens)]
+    need = sum((t + 15) // 16 for t in totals)
+    if num_blocks is None:
+        num_blocks = max(64, 2 * need)
+    if table_width is None:
+        table_width = max(1, max((t + 15) // 16 for t in totals) if totals else 1)
+    return PrefillCase(name=name, seed=seed, num_blocks=num_blocks, num_heads=num_heads,
+                       num_kv_heads=num_kv_heads, head_dim=128, dtype="bf16", scale=128 ** -0.5,
+                       free_order=rng.permutation(num_blocks).astype(np.int32),
+                       ctx_lens=[int(c) for c in ctx_lens], query_lens=[int(n) for n in query_lens],
+                       table_width=table_width)
+
+
+def prefill_case(seed: int = 0, batch: int = 64) -> PrefillCase:
+    """Whole prompts: `batch` prompts with lengths uniform in [16, 1024] (the
+    trace's prompt distribution), Llama-3-8B-shaped heads (32 / 8, head_dim
+    128, bf16), random placement in a 16384-block pool."""
+    rng = np.random.default_rng(seed + 808)
+    n = rng.integers(16, 1024, size=batch, endpoint=True)
+    return PrefillCase(name="prefill_gqa", seed=seed, num_blocks=16384, num_heads=32, num_kv_heads=8,
+                       head_dim=128, dtype="bf16", scale=128 ** -0.5,
+                       free_order=rng.permutation(16384).astype(np.int32),
+                       ctx_lens=[0] * batch, query_lens=[int(x) for x in n], table_width=64)
+
+
+def chunked_prefill_case(seed: int = 0, batch: int = 64, chunk: int = 512) -> PrefillCase:
+    """Chunked prefill: `batch` sequences with cached context uniform in
+    [0, 3072] each bring a chunk of `chunk` new prompt tokens; heads and pool
+    as prefill_case (32768 blocks)."""
+    rng = np.random.default_rng(seed + 909)
+    ctx = rng.integers(0, 3072, size=batch, endpoint=True)
+    return PrefillCase(name="chunked_prefill_gqa", seed=seed, num_blocks=32768, num_heads=32,
+                       num_kv_heads=8, head_dim=128, dtype="bf16", scale=128 ** -0.5,
+                       free_order=rng.permutation(32768).astype(np.int32),
+                       ctx_lens=[int(x) for x in ctx], query_lens=[chunk] * batch,
+                       table_width=(3072 + chunk + 15) // 16)
 
 
 # ---------------------------------------------------------------------------

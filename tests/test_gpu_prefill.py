@@ -1,0 +1,203 @@
+"""GPU parity of paged prefill / chunked prefill (pa_reshape_and_cache of the
+new tokens, then pa_prefill, through the C ABI) against the fp64 oracle on the
+same seeded inputs.
+
+Bars: slot mappings, tables and the appended pool bit-exact; attention
+|err| <= 1e-2 + 2^-8 |ref| (bf16 storage of the result), fp32 accumulation.
+"""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_400_b200 as pk
+from paged_kv_cache_400_b200 import workloads as wl
+from paged_kv_cache_400_b200.scenario import prepare_prefill_step
+
+from oracle_side import (oracle_prefill_all, oracle_prefill_indices, oracle_prefill_rows,
+                         prefill_tolerance_ok, storage_bits)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def device_prefill(case, prep, pool=None):
+    if pool is None:
+        pool = case.make_pool(DEV)
+    q = case.make_q(DEV)
+    k, v = case.make_kv_new(DEV)
+    if case.num_tokens:
+        pk.pa_reshape_and_cache(k, v, pool, torch.from_numpy(prep.slot_mapping).to(DEV))
+    out = torch.zeros_like(q)
+    pk.pa_prefill(out, q, pool, torch.from_numpy(prep.block_tables).to(DEV),
+                  torch.from_numpy(prep.seq_lens).to(DEV), torch.from_numpy(prep.query_start).to(DEV),
+                  case.scale, case.max_query_len)
+    torch.cuda.synchronize()
+    return pool, out
+
+
+def check_indices(case, prep, ost):
+    assert prep.slot_mapping.tolist() == ost.slots
+    assert prep.seq_lens.tolist() == ost.lens
+    for b, tab in enumerate(ost.tables):
+        assert prep.block_tables[b, :len(tab)].tolist() == tab
+
+
+def check_full(case):
+    prep = prepare_prefill_step(case)
+    ost = oracle_prefill_indices(case)
+    check_indices(case, prep, ost)
+    pool, out = device_prefill(case, prep)
+    assert pk.pa_get_device_error() == 0
+    ref, ref_pool = oracle_prefill_all(case, ost)
+    assert np.array_equal(storage_bits(pool), ref_pool)
+    ok, err, worst = prefill_tolerance_ok(out.float().cpu().numpy(), ref)
+    assert ok, f"{case.name}: max|err| {err}, worst err/bar {worst}"
+    return err
+
+
+def test_whole_prompts_ragged():
+    # lengths across tile and block boundaries: 1, 15, 16, 17, 64, 65, 100, 129
+    case = wl.prefill_custom("prompts", 1, [0] * 8, [1, 15, 16, 17, 64, 65, 100, 129], 32, 8)
+    check_full(case)
+
+
+def test_chunked_with_context():
+    case = wl.prefill_custom("chunks", 2, [0, 5, 16, 33, 200, 1], [7, 64, 1, 100, 65, 16], 32, 8)
+    check_full(case)
+
+
+@pytest.mark.parametrize("heads", [(8, 8), (8, 4), (8, 2), (8, 1), (16, 1)])
+def test_head_groups(heads):
+    H, Hkv = heads
+    case = wl.prefill_custom(f"g{H // Hkv}", 3, [0, 40, 3], [70, 33, 130], H, Hkv)
+    check_full(case)
+
+
+def test_empty_sequences_mixed():
+    case = wl.prefill_custom("empty", 4, [0, 20, 0, 17], [0, 0, 37, 0], 32, 8)
+    prep = prepare_prefill_step(case)
+    pool, out = device_prefill(case, prep)
+    assert pk.pa_get_device_error() == 0
+    ost = oracle_prefill_indices(case)
+    ref, _ = oracle_prefill_all(case, ost)
+    ok, err, _ = prefill_tolerance_ok(out.float().cpu().numpy(), ref)
+    assert ok, err
+
+
+def test_nothing_to_do():
+    pool = torch.zeros((4, 2, 8, 16, 128), dtype=torch.bfloat16, device=DEV)
+    q = torch.zeros((0, 32, 128), dtype=torch.bfloat16, device=DEV)
+    z = torch.zeros((0,), dtype=torch.int32, device=DEV)
+    pk.pa_prefill(q, q, pool, torch.zeros((0, 1), dtype=torch.int32, device=DEV), z,
+                  torch.zeros((1,), dtype=torch.int32, device=DEV), 0.1, 0)
+    torch.cuda.synchronize()
+    assert pk.pa_get_device_error() == 0
+
+
+def test_max_group_long_prompt():
+    # one 2000-token prompt with G = 16 (4-token tiles: 500 CTAs on one sequence)
+    case = wl.prefill_custom("long_g16", 5, [0], [2000], 16, 1)
+    prep = prepare_prefill_step(case)
+    ost = oracle_prefill_indices(case)
+    check_indices(case, prep, ost)
+    pool, out = device_prefill(case, prep)
+    assert pk.pa_get_device_error() == 0
+    picks = [(0, i) for i in (0, 1, 2, 3, 15, 16, 17, 511, 1024, 1999)]
+    ref = oracle_prefill_rows(case, ost, picks)
+    got = np.stack([out[i].float().cpu().numpy() for _, i in picks])
+    ok, err, _ = prefill_tolerance_ok(got, ref)
+    assert ok, err
+
+
+def _sampled(case, n_random, seed):
+    prep = prepare_prefill_step(case)
+    ost = oracle_prefill_indices(case)
+    check_indices(case, prep, ost)
+    pool, out = device_prefill(case, prep)
+    assert pk.pa_get_device_error() == 0
+    rng = np.random.default_rng(seed)
+    longest = int(np.argmax(case.query_lens))
+    picks = [(longest, 0), (longest, case.query_lens[longest] - 1), (0, 0),
+             (len(case.query_lens) - 1, case.query_lens[-1] - 1)]
+    for _ in range(n_random):
+        b = int(rng.integers(len(case.query_lens)))
+        picks.append((b, int(rng.integers(case.query_lens[b]))))
+    ref = oracle_prefill_rows(case, ost, picks)
+    starts = prep.query_start
+    got = np.stack([out[int(starts[b]) + i].float().cpu().numpy() for b, i in picks])
+    ok, err, _ = prefill_tolerance_ok(got, ref)
+    assert ok, err
+
+
+def test_prefill_full_size_sampled():
+    _sampled(wl.prefill_case(0), 24, 0)
+
+
+def test_chunked_prefill_full_size_sampled():
+    _sampled(wl.chunked_prefill_case(0), 24, 1)
+
+
+def test_last_row_matches_decode():
+    # the newest token's prefill row attends to the whole sequence, as decode does
+    case = wl.prefill_custom("vs_decode", 6, [100, 0, 31], [50, 77, 1], 32, 8)
+    prep = prepare_prefill_step(case)
+    pool, out = device_prefill(case, prep)
+    last = torch.from_numpy(prep.query_start[1:] - 1).long().to(DEV)
+    q = case.make_q(DEV)[last].contiguous()
+    dec = torch.empty_like(q)
+    bt = torch.from_numpy(prep.block_tables).to(DEV)
+    sl = torch.from_numpy(prep.seq_lens).to(DEV)
+    ws = pk.alloc_workspace(3, 32, pool, int(prep.seq_lens.max()))
+    pk.pa_decode(dec, q, pool, bt, sl, case.scale, int(prep.seq_lens.max()), ws)
+    torch.cuda.synchronize()
+    assert pk.pa_get_device_error() == 0
+    assert (dec.float() - out[last].float()).abs().max().item() <= 1e-2
+
+
+def test_bad_lengths_flagged():
+    case = wl.prefill_custom("bad", 7, [0, 0], [20, 20], 32, 8)
+    prep = prepare_prefill_step(case)
+    pool = case.make_pool(DEV)
+    before = pool.clone()
+    q = case.make_q(DEV)
+    out = torch.zeros_like(q)
+    sl = torch.tensor([20, 10], dtype=torch.int32, device=DEV)   # n = 20 > L = 10
+    pk.pa_prefill(out, q, pool, torch.from_numpy(prep.block_tables).to(DEV), sl,
+                  torch.from_numpy(prep.query_start).to(DEV), case.scale, case.max_query_len)
+    torch.cuda.synchronize()
+    assert pk.pa_get_device_error() == pk.PA_DEVERR_SEQLEN
+    assert torch.equal(pool, before)
+    assert out[20:].abs().max().item() == 0.0   # the bad sequence is skipped
+
+
+def test_bad_block_flagged():
+    # block 1 of the table (positions 16..31) points outside the pool: flagged,
+    # never read; the first 16-token tile (32 / 8 heads: 16 tokens) reads
+    # block 0 only and stays exact
+    case = wl.prefill_custom("badblk", 8, [0], [40], 32, 8)
+    prep = prepare_prefill_step(case)
+    pool = case.make_pool(DEV)
+    k, v = case.make_kv_new(DEV)
+    pk.pa_reshape_and_cache(k, v, pool, torch.from_numpy(prep.slot_mapping).to(DEV))
+    bt = prep.block_tables.copy()
+    bt[0, 1] = case.num_blocks + 5
+    q = case.make_q(DEV)
+    out = torch.zeros_like(q)
+    pk.pa_prefill(out, q, pool, torch.from_numpy(bt).to(DEV), torch.from_numpy(prep.seq_lens).to(DEV),
+                  torch.from_numpy(prep.query_start).to(DEV), case.scale, case.max_query_len)
+    torch.cuda.synchronize()
+    assert pk.pa_get_device_error() == pk.PA_DEVERR_BLOCK
+    ost = oracle_prefill_indices(case)
+    ref = oracle_prefill_rows(case, ost, [(0, i) for i in range(16)])
+    ok, err, _ = prefill_tolerance_ok(out[:16].float().cpu().numpy(), ref)
+    assert ok, err
+    assert torch.isfinite(out.float()).all()
+
+
+def test_unsupported_rejected():
+    pool = torch.zeros((4, 2, 3, 16, 128), dtype=torch.bfloat16, device=DEV)
+    q = torch.zeros((1, 9, 128), dtype=torch.bfloat16, device=DEV)  # G = 3
+    one = torch.ones((1,), dtype=torch.int32, device=DEV)
+    qs = torch.tensor([0, 1], dtype=torch.int32, device=DEV)
+    with pytest.raises(pk.PagedKVError):
+        pk.pa_prefill(q, q, pool, torch.zeros((1, 1), dtype=torch.int32, device=DEV), one, qs, 0.1, 1)
