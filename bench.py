@@ -697,6 +697,7 @@ def run_prefill(args, rank, world, dist):
     if rank != 0:
         return
     flops = prefill_flops(case)
+    mma_sync = os.environ.get("PAGEDKV_PREFILL_KERNEL") == "mma_sync"
     att_avg = sum(att_ms) / K
     peak, peak_src = measured_tensor_peak()
     achieved = flops / (att_avg / 1e3) / 1e12
@@ -716,11 +717,12 @@ def run_prefill(args, rank, world, dist):
                    "parallelism": f"dp{world} independent replicas (no exchange step)",
                    "l2": "no flush: K/V read %.2f GB per step (> 126 MB L2), q/out %.2f GB"
                          % (kv_bytes / 1e9, 2 * T * case.num_heads * case.head_dim * 2 / 1e9)},
-        "roofline": {"kernel": "prefill_kernel (pa_prefill)", "bound": "tensor", "achieved": achieved,
+        "roofline": {"kernel": ("prefill_kernel (mma.sync m16n8k16)" if mma_sync else
+                                "prefill_tc_kernel (tcgen05.mma, accumulators in tensor memory)"),
+                     "bound": "tensor", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_src,
                      "traffic": None, "traffic_source": "not captured on this source",
-                     "algorithmic_flops_per_launch": flops, "avg_launch_ms": att_avg,
-                     "note": "mma.sync m16n8k16 (legacy tensor path on sm_100a)"},
+                     "algorithmic_flops_per_launch": flops, "avg_launch_ms": att_avg},
         "append_avg_ms": sum(app_ms) / K,
         "gpu_launches": 2 * K,
         "clocks": sampler.summary(wall0, wall1),

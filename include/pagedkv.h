@@ -241,7 +241,9 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* kv_pool,
  * n_b > seq_lens[b] or seq_lens[b] > 16 * max_blocks_per_seq sets
  * PA_DEVERR_SEQLEN and skips sequence b; a block id outside the pool sets
  * PA_DEVERR_BLOCK (that block's contribution is undefined, nothing is read
- * from it). Allocates nothing.
+ * from it). A wait on staged data that exceeds 2 s sets PA_DEVERR_TIMEOUT; while
+ * that bit is set (until pa_get_device_error reads it), prefill tiles that
+ * start later skip their work. Allocates nothing.
  */
 pa_status pa_prefill(void* out, const void* q, const void* kv_pool,
                      const int32_t* block_tables, int32_t max_blocks_per_seq,

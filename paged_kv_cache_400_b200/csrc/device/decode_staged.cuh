@@ -546,14 +546,16 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Tensor map of a bf16 head_dim-128 pool: (d 128, row 16, kv head, K|V, block),
-// box (64, 16, 1, 2, 1), 128-byte swizzle, zero fill outside the tensor.
-inline pa_status encode_pool_map(const void* pool, int32_t num_kv_heads, int32_t num_blocks, CUtensorMap* map) {
+// box (64, 16, 1, box_kv, 1) -- K and V of a block together (box_kv 2) or one of
+// them (box_kv 1) -- 128-byte swizzle, zero fill outside the tensor.
+inline pa_status encode_pool_map(const void* pool, int32_t num_kv_heads, int32_t num_blocks, CUtensorMap* map,
+                                 uint32_t box_kv = 2) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const cuuint64_t hkv = (cuuint64_t)num_kv_heads;
   const cuuint64_t dims[5] = {128, 16, hkv, 2, (cuuint64_t)num_blocks};
   const cuuint64_t strides[4] = {256, 4096, hkv * 4096, 2 * hkv * 4096};
-  const cuuint32_t box[5] = {64, 16, 1, 2, 1};
+  const cuuint32_t box[5] = {64, 16, 1, box_kv, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(pool), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

@@ -2,6 +2,7 @@
 // launches. All kernels live in this one translation unit so they share the
 // per-device error word without relocatable device code.
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -12,6 +13,7 @@
 #include "decode_generic.cuh"
 #include "decode_staged.cuh"
 #include "prefill.cuh"
+#include "prefill_tc.cuh"
 
 using pagedkv::fail;
 
@@ -350,7 +352,15 @@ pa_status pa_prefill(void* out, const void* q, const void* kv_pool, const int32_
   p.max_query_len = max_query_len;
   p.num_tokens = num_tokens;
   p.scale_log2 = scale * pagedkv::kLog2e;
-  return pagedkv::launch_prefill_bf16_d128(kv_pool, pool.num_blocks, p, num_seqs, (cudaStream_t)stream);
+  // tcgen05 kernel; PAGEDKV_PREFILL_KERNEL=mma_sync selects the mma.sync kernel
+  // (same results within rounding; kept for comparison)
+  const char* which = std::getenv("PAGEDKV_PREFILL_KERNEL");
+  if (which && std::strcmp(which, "mma_sync") == 0) {
+    p.tile_tokens = 64 / G;
+    return pagedkv::launch_prefill_bf16_d128(kv_pool, pool.num_blocks, p, num_seqs, (cudaStream_t)stream);
+  }
+  p.tile_tokens = 128 / G;
+  return pagedkv::launch_prefill_tc(kv_pool, pool.num_blocks, p, num_seqs, (cudaStream_t)stream);
 }
 
 pa_status pa_copy_blocks(void* kv_pool, const int32_t* src, const int32_t* dst, int32_t n,

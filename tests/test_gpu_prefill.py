@@ -20,6 +20,17 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
+@pytest.fixture(autouse=True, params=["tcgen05", "mma_sync"])
+def prefill_kernel(request, monkeypatch):
+    """Every test runs on both prefill kernels (tcgen05 is the default;
+    PAGEDKV_PREFILL_KERNEL=mma_sync selects the mma.sync one)."""
+    if request.param == "mma_sync":
+        monkeypatch.setenv("PAGEDKV_PREFILL_KERNEL", "mma_sync")
+    else:
+        monkeypatch.delenv("PAGEDKV_PREFILL_KERNEL", raising=False)
+    return request.param
+
+
 def device_prefill(case, prep, pool=None):
     if pool is None:
         pool = case.make_pool(DEV)
@@ -172,8 +183,7 @@ def test_bad_lengths_flagged():
 
 def test_bad_block_flagged():
     # block 1 of the table (positions 16..31) points outside the pool: flagged,
-    # never read; the first 16-token tile (32 / 8 heads: 16 tokens) reads
-    # block 0 only and stays exact
+    # never read; rows 0..15 attend to block 0 only and stay exact
     case = wl.prefill_custom("badblk", 8, [0], [40], 32, 8)
     prep = prepare_prefill_step(case)
     pool = case.make_pool(DEV)
