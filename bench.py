@@ -60,6 +60,8 @@ def parse_args():
                     help="trace: replay each step's decode over all layers as a CUDA graph")
     ap.add_argument("--batch", type=int, default=256,
                     help="sequences per GPU (256 is the workload; smaller only for profiling captures)")
+    ap.add_argument("--prefill-batch", type=int, default=64,
+                    help="prefill workloads: sequences per GPU (64 is the workload; smaller for captures)")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bounded oracle sample for cpu_baseline")
@@ -634,7 +636,9 @@ def run_prefill(args, rank, world, dist):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     chunked = args.workload == "chunked_prefill"
-    case = (wl.chunked_prefill_case(args.seed + rank) if chunked else wl.prefill_case(args.seed + rank))
+    pb = args.prefill_batch
+    case = (wl.chunked_prefill_case(args.seed + rank, batch=pb) if chunked
+            else wl.prefill_case(args.seed + rank, batch=pb))
     prep = prepare_prefill_step(case)
     T = case.num_tokens
     pool = case.make_pool(dev)
@@ -703,8 +707,8 @@ def run_prefill(args, rank, world, dist):
     achieved = flops / (att_avg / 1e3) / 1e12
     kv_bytes = int(sum(int(c) + int(n) for c, n in zip(case.ctx_lens, case.query_lens))) * 2 * \
         case.num_kv_heads * case.head_dim * 2
-    desc = ("chunked_prefill_gqa: 64 sequences, cached context U[0,3072] + a 512-token chunk"
-            if chunked else "prefill_gqa: 64 whole prompts, lengths U[16,1024]")
+    desc = (f"chunked_prefill_gqa: {pb} sequences, cached context U[0,3072] + a 512-token chunk"
+            if chunked else f"prefill_gqa: {pb} whole prompts, lengths U[16,1024]")
     line = {
         "metric": "paged prefill new tokens/s (append + causal paged attention)", "value": value,
         "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,

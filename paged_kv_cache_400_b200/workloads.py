@@ -345,24 +345,26 @@ def prefill_custom(name, seed, ctx_lens, query_lens, num_heads=32, num_kv_heads=
 def prefill_case(seed: int = 0, batch: int = 64) -> PrefillCase:
     """Whole prompts: `batch` prompts with lengths uniform in [16, 1024] (the
     trace's prompt distribution), Llama-3-8B-shaped heads (32 / 8, head_dim
-    128, bf16), random placement in a 16384-block pool."""
+    128, bf16), random placement in a 256 x batch-block pool (16384 at 64)."""
     rng = np.random.default_rng(seed + 808)
     n = rng.integers(16, 1024, size=batch, endpoint=True)
-    return PrefillCase(name="prefill_gqa", seed=seed, num_blocks=16384, num_heads=32, num_kv_heads=8,
+    nb = 256 * batch
+    return PrefillCase(name="prefill_gqa", seed=seed, num_blocks=nb, num_heads=32, num_kv_heads=8,
                        head_dim=128, dtype="bf16", scale=128 ** -0.5,
-                       free_order=rng.permutation(16384).astype(np.int32),
+                       free_order=rng.permutation(nb).astype(np.int32),
                        ctx_lens=[0] * batch, query_lens=[int(x) for x in n], table_width=64)
 
 
 def chunked_prefill_case(seed: int = 0, batch: int = 64, chunk: int = 512) -> PrefillCase:
     """Chunked prefill: `batch` sequences with cached context uniform in
-    [0, 3072] each bring a chunk of `chunk` new prompt tokens; heads and pool
-    as prefill_case (32768 blocks)."""
+    [0, 3072] each bring a chunk of `chunk` new prompt tokens; heads as
+    prefill_case, a 512 x batch-block pool (32768 at 64)."""
     rng = np.random.default_rng(seed + 909)
     ctx = rng.integers(0, 3072, size=batch, endpoint=True)
-    return PrefillCase(name="chunked_prefill_gqa", seed=seed, num_blocks=32768, num_heads=32,
+    nb = 512 * batch
+    return PrefillCase(name="chunked_prefill_gqa", seed=seed, num_blocks=nb, num_heads=32,
                        num_kv_heads=8, head_dim=128, dtype="bf16", scale=128 ** -0.5,
-                       free_order=rng.permutation(32768).astype(np.int32),
+                       free_order=rng.permutation(nb).astype(np.int32),
                        ctx_lens=[int(x) for x in ctx], query_lens=[chunk] * batch,
                        table_width=(3072 + chunk + 15) // 16)
 

@@ -20,14 +20,17 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-@pytest.fixture(autouse=True, params=["tcgen05", "mma_sync"])
+@pytest.fixture(autouse=True, params=["tcgen05", "tcgen05_1tile", "mma_sync"])
 def prefill_kernel(request, monkeypatch):
-    """Every test runs on both prefill kernels (tcgen05 is the default;
-    PAGEDKV_PREFILL_KERNEL=mma_sync selects the mma.sync one)."""
+    """Every test runs on each prefill kernel: tcgen05 with two query tiles per
+    CTA (the default), tcgen05 with one (PAGEDKV_PREFILL_QTILES=1), and the
+    mma.sync kernel (PAGEDKV_PREFILL_KERNEL=mma_sync)."""
+    monkeypatch.delenv("PAGEDKV_PREFILL_KERNEL", raising=False)
+    monkeypatch.delenv("PAGEDKV_PREFILL_QTILES", raising=False)
     if request.param == "mma_sync":
         monkeypatch.setenv("PAGEDKV_PREFILL_KERNEL", "mma_sync")
-    else:
-        monkeypatch.delenv("PAGEDKV_PREFILL_KERNEL", raising=False)
+    elif request.param == "tcgen05_1tile":
+        monkeypatch.setenv("PAGEDKV_PREFILL_QTILES", "1")
     return request.param
 
 
