@@ -195,27 +195,32 @@ class ClockSampler:
 DECODE_KERNEL_SOURCES = ("common.cuh", "decode_common.cuh", "decode_staged.cuh", "ptx.cuh")
 
 
-def kernel_source_digest():
-    """Digest of the sources the staged decode kernel is compiled from."""
+PREFILL_KERNEL_SOURCES = ("common.cuh", "ptx.cuh", "tcgen05.cuh", "decode_common.cuh", "decode_staged.cuh",
+                          "prefill.cuh", "prefill_tc.cuh")
+
+
+def kernel_source_digest(sources=None):
+    """Digest of the sources a kernel is compiled from (default: the staged
+    decode kernel's)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_400_b200", "csrc", "device")
-    for n in DECODE_KERNEL_SOURCES:
+    for n in (sources or DECODE_KERNEL_SOURCES):
         with open(os.path.join(csrc, n), "rb") as f:
             h.update(n.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic():
+def recorded_traffic(path=None, sources=None):
     """ncu DRAM bytes per launch recorded in profiles/, if taken on this source."""
     try:
-        text = open(TRAFFIC_FILE).read()
+        text = open(path or TRAFFIC_FILE).read()
     except OSError:
         return None, "no ncu summary"
     m = re.search(r"kernel_source_digest:\s*([0-9a-f]+)", text)
     t = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
     if not (m and t):
         return None, "summary lacks digest or traffic"
-    if m.group(1) != kernel_source_digest():
+    if m.group(1) != kernel_source_digest(sources):
         return None, "kernel changed since the ncu capture"
     return int(t.group(1)), "ncu capture"
 
@@ -707,6 +712,12 @@ def run_prefill(args, rank, world, dist):
     achieved = flops / (att_avg / 1e3) / 1e12
     kv_bytes = int(sum(int(c) + int(n) for c, n in zip(case.ctx_lens, case.query_lens))) * 2 * \
         case.num_kv_heads * case.head_dim * 2
+    traffic, traffic_src = None, ("mma.sync kernel: not captured" if mma_sync else
+                                  "captured at 64 sequences only")
+    if not mma_sync and pb == 64:
+        traffic, traffic_src = recorded_traffic(
+            os.path.join(ROOT, "profiles", f"prefill_tc_{'chunked' if chunked else 'prompts'}_b64.md"),
+            PREFILL_KERNEL_SOURCES)
     desc = (f"chunked_prefill_gqa: {pb} sequences, cached context U[0,3072] + a 512-token chunk"
             if chunked else f"prefill_gqa: {pb} whole prompts, lengths U[16,1024]")
     line = {
@@ -725,7 +736,8 @@ def run_prefill(args, rank, world, dist):
                                 "prefill_tc_kernel (tcgen05.mma, accumulators in tensor memory)"),
                      "bound": "tensor", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_src,
-                     "traffic": None, "traffic_source": "not captured on this source",
+                     "traffic": traffic, "traffic_source": traffic_src,
+                     "algorithmic_kv_bytes": kv_bytes,
                      "algorithmic_flops_per_launch": flops, "avg_launch_ms": att_avg},
         "append_avg_ms": sum(app_ms) / K,
         "gpu_launches": 2 * K,

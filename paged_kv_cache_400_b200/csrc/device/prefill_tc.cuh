@@ -55,9 +55,9 @@ constexpr float kTcRescaleLog2 = 8.0f;            // raise the reference max pas
 template <int kQTiles>
 struct TcConfig {
   static constexpr int kStages = kQTiles == 2 ? 4 : 2;
-  static constexpr int kThreads = kQTiles * 128 + 64;
+  static constexpr int kThreads = kQTiles * 128 + 32 + kQTiles * 32;
   static constexpr int kProducerWarp = kQTiles * 4;
-  static constexpr int kMmaWarp = kQTiles * 4 + 1;
+  static constexpr int kMmaWarp = kQTiles * 4 + 1;  // first of kQTiles issuer warps, one per tile
   static constexpr uint32_t kTmemCols = kQTiles * 256;
   static constexpr int kSmem = kQTiles * kTcQBytes + kStages * kTcStageBytes + 1024;
 };
@@ -68,7 +68,7 @@ struct PrefillTcShared {
   uint64_t kv_full[TcConfig<kQTiles>::kStages];
   uint64_t kv_empty[TcConfig<kQTiles>::kStages];
   uint64_t s_full[kQTiles][2];   // S_j of tile t ready: s_full[t][j & 1]
-  uint64_t p_full[kQTiles][2];   // P_j of tile t written (128 arrivals)
+  uint64_t p_full[kQTiles][2];   // P_j of tile t written (one arrival per softmax warp)
   uint64_t pv_done[kQTiles][2];  // PV_j of tile t complete: pv_done[t][j & 1]
   uint32_t tmem_base;
 };
@@ -144,14 +144,14 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
 #pragma unroll
     for (int s = 0; s < S; ++s) {
       mbar_init(&sh.kv_full[s], 1);
-      mbar_init(&sh.kv_empty[s], 1);
+      mbar_init(&sh.kv_empty[s], kQTiles);  // one release per issuer
     }
 #pragma unroll
     for (int t = 0; t < kQTiles; ++t)
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         mbar_init(&sh.s_full[t][i], 1);
-        mbar_init(&sh.p_full[t][i], 128);
+        mbar_init(&sh.p_full[t][i], 4);  // one arrival per softmax warp
         mbar_init(&sh.pv_done[t][i], 1);
       }
     fence_barrier_init();
@@ -244,27 +244,31 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
         }
       }
     }
-  } else if (warp == Cfg::kMmaWarp) {
-    // ---- MMA issuer ----------------------------------------------------------------
+  } else if (warp >= Cfg::kMmaWarp) {
+    // ---- MMA issuers: warp kMmaWarp + t, one thread, drives query tile t -------------
+    const int t = warp - Cfg::kMmaWarp;
+    const int32_t ntt = (kQTiles == 1 || t == 0) ? nt[0] : nt[kQTiles - 1];
     if (lane == 0) {
       constexpr uint32_t idesc_s = tc_idesc_bf16(128, kTcKeys, false);
       constexpr uint32_t idesc_pv = tc_idesc_bf16(128, 128, true);
-      const uint32_t q_addr = smem_addr(q_smem);
+      const uint32_t qa = smem_addr(q_smem) + t * kTcQBytes;
       const uint32_t kv_addr = smem_addr(kv_smem);
+      const uint32_t tm = tmem + t * 256;
       bool ok = mbar_wait_bounded(&sh.q_full, 0, kWaitLimitNs);
-      int32_t kv_ready = -1;  // KV tiles 0 .. kv_ready have been waited for
-      // S_j of tile t = Q_t K_j^T: eight k-steps of 16 dims (32 bytes inside the
-      // swizzled 128-byte rows; dims 64..127 in the second half region).
-      auto issue_s = [&](int t, int32_t j) {
-        if (j > kv_ready) {
-          ok = ok && mbar_wait_bounded(&sh.kv_full[j % S], (uint32_t)(j / S) & 1u, kWaitLimitNs);
-          kv_ready = j;
-        }
+      int32_t kv_ready = -1;  // KV tiles 0 .. kv_ready have been waited for, in order
+      auto ensure_kv = [&](int32_t j) {
+        for (int32_t i = kv_ready + 1; i <= j && ok; ++i)
+          ok = mbar_wait_bounded(&sh.kv_full[i % S], (uint32_t)(i / S) & 1u, kWaitLimitNs);
+        kv_ready = j;
+      };
+      // S_j = Q_t K_j^T: eight k-steps of 16 dims (32 bytes inside the swizzled
+      // 128-byte rows; dims 64..127 in the second half region).
+      auto issue_s = [&](int32_t j) {
+        ensure_kv(j);
         if (!ok) return;
         tc_fence_after_sync();
-        const uint32_t qa = q_addr + t * kTcQBytes;
         const uint32_t kaddr = kv_addr + (j % S) * kTcStageBytes;
-        const uint32_t d = tmem + t * 256 + 128 + 64 * (j & 1);
+        const uint32_t d = tm + 128 + 64 * (j & 1);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * (kTcQBytes / 2) + (kk & 3) * 32;
@@ -274,14 +278,10 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
         }
         tc_commit(&sh.s_full[t][j & 1]);
       };
-#pragma unroll
-      for (int t = 0; t < kQTiles; ++t)
-        if (ok && nt[t] > 0) issue_s(t, 0);
+      if (ok && ntt > 0) issue_s(0);
       for (int32_t j = 0; j < nt_max && ok; ++j) {
-#pragma unroll
-        for (int t = 0; t < kQTiles; ++t) {
-          if (j >= nt[t]) continue;
-          if (j + 1 < nt[t]) issue_s(t, j + 1);
+        if (j < ntt) {
+          if (j + 1 < ntt) issue_s(j + 1);
           ok = ok && mbar_wait_bounded(&sh.p_full[t][j & 1], (uint32_t)(j >> 1) & 1u, kWaitLimitNs);
           if (!ok) break;
           tc_fence_after_sync();
@@ -289,14 +289,18 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
           // contiguous), its two 64-dim halves one leading offset apart, 8-key
           // groups 1024 B apart.
           const uint32_t vaddr = kv_addr + (j % S) * kTcStageBytes + tc_region(1, 0);
-          const uint32_t pa = tmem + t * 256 + 128 + 64 * (j & 1);
+          const uint32_t pa = tm + 128 + 64 * (j & 1);
 #pragma unroll
           for (int kk = 0; kk < kTcKeys / 16; ++kk)
-            tc_mma_ts(tmem + t * 256, pa + 8 * kk, tc_desc_sw128(vaddr + kk * 2048, kTcHalfBytes, 1024), idesc_pv,
+            tc_mma_ts(tm, pa + 8 * kk, tc_desc_sw128(vaddr + kk * 2048, kTcHalfBytes, 1024), idesc_pv,
                       (j > 0 || kk > 0) ? 1u : 0u);
           tc_commit(&sh.pv_done[t][j & 1]);
+          if (j + S < nt_max) tc_commit(&sh.kv_empty[j % S]);
+        } else if (j + S < nt_max) {
+          // this tile never reads KV tile j; release it in order, after its load
+          ensure_kv(j);
+          if (ok) mbar_arrive(&sh.kv_empty[j % S]);
         }
-        if (ok && j + S < nt_max) tc_commit(&sh.kv_empty[j % S]);
       }
       if (!ok) raise_device_error(PA_DEVERR_TIMEOUT);
     }
@@ -385,7 +389,8 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
       tmem_st32(sbuf, pw);
       tmem_wait_st();
       tc_fence_before_sync();
-      mbar_arrive(&sh.p_full[t][j & 1]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.p_full[t][j & 1]);
     }
     if (ok && ntt > 0) {
       const bool done =
