@@ -81,15 +81,6 @@ __device__ __forceinline__ float ex2_sfu(float x) {
   return y;
 }
 
-// Two non-negative finite floats to a packed bf16 pair, round to nearest even
-// (adding 0x7FFF plus the kept lowest bit before truncation) with integer ops.
-__device__ __forceinline__ uint32_t pack_bf16x2_nonneg(float lo, float hi) {
-  uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
-  a += 0x7FFFu + ((a >> 16) & 1u);
-  b += 0x7FFFu + ((b >> 16) & 1u);
-  return __byte_perm(a, b, 0x7632);
-}
-
 // Region offsets inside a stage.
 __device__ __forceinline__ uint32_t tc_region(int kv, int half) { return (uint32_t)((kv * 2 + half) * kTcHalfBytes); }
 
@@ -383,7 +374,7 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
           p1 = key0 + 2 * c + 1 <= P ? p1 : 0.f;
         }
         sum += p0 + p1;
-        pw[c] = pack_bf16x2_nonneg(p0, p1);
+        pw[c] = pack_bf16x2(p0, p1);
       }
       l += sum;
       tmem_st32(sbuf, pw);
