@@ -56,6 +56,8 @@ def parse_args():
                     help="trace: pinned host blocks per layer for swap-mode preemption (0: recompute)")
     ap.add_argument("--no-prefix-cache", action="store_true",
                     help="prefix_trace: run without automatic prefix caching (for comparison)")
+    ap.add_argument("--prefill", action="store_true",
+                    help="trace: also run the admitted prompts' causal prefill attention (pa_prefill) per layer")
     ap.add_argument("--graphs", action="store_true",
                     help="trace: replay each step's decode over all layers as a CUDA graph")
     ap.add_argument("--batch", type=int, default=256,
@@ -530,7 +532,7 @@ def run_trace(args, rank, world):
         if n:
             reqs_p, pos_p = eng.prompt_positions(idx)
             inputs, stacked = tr.step_inputs(idx.step, idx.running, idx.seq_lens, reqs_p, pos_p, dev,
-                                             stacked=True)
+                                             stacked=True, prefill=args.prefill)
             if graphed is not None:
                 graphed._graph(((n + graphed.bucket - 1) // graphed.bucket) * graphed.bucket)
             torch.cuda.synchronize()
@@ -565,10 +567,13 @@ def run_trace(args, rank, world):
                else "prompts U[16,1024]")
     line = {
         "graphs": bool(args.graphs),
+        "prefill_attention": bool(args.prefill),
         "prefix_caching": caching,
         "workload": f"continuous-batching trace: {args.trace_requests} requests, Poisson(50) arrivals/step, "
                     f"{prompts}, outputs geometric mean 200 cap 2048, 40000-block pools, "
-                    f"{tr.num_layers} layers x (prompt append + decode-token append + paged decode), "
+                    f"{tr.num_layers} layers x (prompt append + "
+                    + ("causal prefill attention of the new prompt positions + " if args.prefill else "")
+                    + "decode-token append + paged decode), "
                     "32/8 heads, head_dim 128, bf16",
         "prompt_tokens_cached": cached_tokens, "peak_batch": peak_batch,
         "swap_host_blocks": args.swap_host_blocks,

@@ -15,7 +15,8 @@
 //              r of its tile = tensor-memory lane r;
 //   warp 8     producer: both Q tiles by TMA once, then KV tiles of 64 keys
 //              (four 16-token blocks gathered through the table, one TMA box
-//              per block and K|V and head-dim half) into a 4-stage ring;
+//              per block and K|V and head-dim half, the 16 boxes issued by 16
+//              lanes at once) into a 4-stage ring;
 //   warp 9     MMA issuer (one thread): per tile, S = Q K^T into tensor
 //              memory, then O += P V with P read back from tensor memory.
 // Tensor memory (512 columns, so one CTA per SM): per tile t at 256 t, O
@@ -40,6 +41,8 @@
 #include "decode_staged.cuh"
 #include "tcgen05.cuh"
 
+#include <cstdlib>
+
 namespace pagedkv {
 
 constexpr int kTcKeys = 64;                       // keys per KV tile
@@ -62,11 +65,11 @@ struct TcConfig {
   static constexpr int kSmem = kQTiles * kTcQBytes + kStages * kTcStageBytes + 1024;
 };
 
-template <int kQTiles>
+template <int kQTiles, int kStages>
 struct PrefillTcShared {
   uint64_t q_full;
-  uint64_t kv_full[TcConfig<kQTiles>::kStages];
-  uint64_t kv_empty[TcConfig<kQTiles>::kStages];
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
   uint64_t s_full[kQTiles][2];   // S_j of tile t ready: s_full[t][j & 1]
   uint64_t p_full[kQTiles][2];   // P_j of tile t written (one arrival per softmax warp)
   uint64_t pv_done[kQTiles][2];  // PV_j of tile t complete: pv_done[t][j & 1]
@@ -91,7 +94,7 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
   using Cfg = TcConfig<kQTiles>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ PrefillTcShared<kQTiles> sh;
+  __shared__ PrefillTcShared<kQTiles, S> sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_smem = smem;
   uint8_t* kv_smem = smem + kQTiles * kTcQBytes;
@@ -168,16 +171,21 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
         tma_load_3d(q_smem + t * kTcQBytes + kTcQBytes / 2, &q_map, &sh.q_full, 64, g * G, q0 + tok_begin + t * QT);
       }
     }
-    // lanes 0..3 hold the block ids of one KV tile; the next tile's ids are
-    // fetched while this one is staged
-    auto load_ids = [&](int32_t j) -> int32_t {
-      const int32_t bi = j * kTcBlocksPerTile + lane;
-      return (lane < kTcBlocksPerTile && bi < nblocks) ? __ldg(table + bi) : -1;
+    // block ids in batches of 32 (8 KV tiles), lane l holding entry l of its
+    // batch; the next batch is in flight while the current one is staged
+    constexpr int32_t kTilesPerBatch = 32 / kTcBlocksPerTile;
+    auto load_batch = [&](int32_t k) -> int32_t {
+      const int32_t bi = k * 32 + lane;
+      return bi < nblocks ? __ldg(table + bi) : -1;
     };
-    int32_t ids_next = load_ids(0);
+    int32_t ids = load_batch(0);
+    int32_t ids_next = load_batch(1);
     for (int32_t j = 0; j < nt_max; ++j) {
-      const int32_t ids = ids_next;
-      if (j + 1 < nt_max) ids_next = load_ids(j + 1);
+      if (j > 0 && j % kTilesPerBatch == 0) {
+        ids = ids_next;
+        ids_next = load_batch(j / kTilesPerBatch + 1);
+      }
+      const int32_t first = (j % kTilesPerBatch) * kTcBlocksPerTile;  // this tile's entries in the batch
       const int32_t s = j % S;
       if (j >= S) {
         const bool ok = mbar_wait_bounded(&sh.kv_empty[s], (uint32_t)(j / S - 1) & 1u, kWaitLimitNs);
@@ -195,7 +203,7 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
 #pragma unroll
       for (int32_t i = 0; i < kTcBlocksPerTile; ++i) {
         const int32_t bi = j * kTcBlocksPerTile + i;
-        blk[i] = __shfl_sync(0xffffffffu, ids, i);
+        blk[i] = __shfl_sync(0xffffffffu, ids, first + i);
         if (bi < nblocks && (blk[i] < 0 || blk[i] >= p.num_blocks)) {
           if (lane == 0) raise_device_error(PA_DEVERR_BLOCK);
           blk[i] = -1;
@@ -217,22 +225,21 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
           *reinterpret_cast<uint4*>(st + tc_region(kv, c >> 3) + key * 128 + (((c & 7) ^ (key & 7)) << 4)) = val;
         }
       }
-      fence_proxy_async_smem();
+      if (tma_mask != (1u << kTcBlocksPerTile) - 1) fence_proxy_async_smem();  // the warp wrote slots
       __syncwarp();
       if (lane == 0) {
         const uint32_t bytes = (uint32_t)__popc(tma_mask) * 4u * 2048u;
         if (bytes) mbar_arrive_expect_tx(&sh.kv_full[s], bytes);
         else mbar_arrive(&sh.kv_full[s]);
-#pragma unroll
-        for (int32_t i = 0; i < kTcBlocksPerTile; ++i) {
-          if (!((tma_mask >> i) & 1u)) continue;
-#pragma unroll
-          for (int kv = 0; kv < 2; ++kv)
-#pragma unroll
-            for (int half = 0; half < 2; ++half)
-              tma_load_5d(st + tc_region(kv, half) + i * 2048, &pool_map, &sh.kv_full[s], 64 * half, 0, g, kv,
-                          blk[i]);
-        }
+      }
+      __syncwarp();
+      // one TMA box per lane: lane = 4 x block slot + 2 x (K|V) + head-dim half
+      const int32_t my_blk = __shfl_sync(0xffffffffu, ids, first + ((lane >> 2) & 3));
+      if (lane < 4 * kTcBlocksPerTile && ((tma_mask >> (lane >> 2)) & 1u)) {
+        const int kv = (lane >> 1) & 1;
+        const int half = lane & 1;
+        tma_load_5d(st + tc_region(kv, half) + (lane >> 2) * 2048, &pool_map, &sh.kv_full[s], 64 * half, 0, g, kv,
+                    my_blk);
       }
     }
   } else if (warp >= Cfg::kMmaWarp) {
@@ -329,8 +336,10 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
           mt = fmaxf(mt, __uint_as_float(sr[c]));
         }
       } else {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent chains
 #pragma unroll
-        for (int c = 0; c < 64; ++c) mt = fmaxf(mt, __uint_as_float(sr[c]));
+        for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c]));
+        mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
       mt *= p.scale_log2;
       if (j == 0) {
@@ -362,7 +371,7 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
       // p = 2^(s * scale - m) on the special-function unit
       const float neg_m = -m_ref;
       uint32_t pw[32];
-      float sum = 0.f;
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         const float x0 = fmaf(__uint_as_float(sr[2 * c]), p.scale_log2, neg_m);
@@ -373,10 +382,10 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
           p0 = key0 + 2 * c <= P ? p0 : 0.f;
           p1 = key0 + 2 * c + 1 <= P ? p1 : 0.f;
         }
-        sum += p0 + p1;
+        sum4[c & 3] += p0 + p1;
         pw[c] = pack_bf16x2(p0, p1);
       }
-      l += sum;
+      l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       tmem_st32(sbuf, pw);
       tmem_wait_st();
       tc_fence_before_sync();
@@ -444,8 +453,8 @@ inline pa_status launch_prefill_tc_variant(const CUtensorMap& pool_map, const CU
                                            const PrefillParams& p, const uint4* pool, int32_t num_seqs,
                                            cudaStream_t st) {
   using Cfg = TcConfig<kQTiles>;
-  static cudaError_t attr =
-      cudaFuncSetAttribute(prefill_tc_kernel<kQTiles>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+  static cudaError_t attr = cudaFuncSetAttribute(prefill_tc_kernel<kQTiles>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
   if (attr != cudaSuccess) return fail(PA_ERR_CUDA, "pa_prefill: %s", cudaGetErrorString(attr));
   const int32_t unit_tokens = kQTiles * (128 / p.group);
   dim3 grid((p.max_query_len + unit_tokens - 1) / unit_tokens, p.num_kv_heads, num_seqs);

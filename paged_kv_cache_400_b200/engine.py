@@ -88,6 +88,7 @@ class DecodeEngine:
             self.host_pools = [torch.empty(hshape, dtype=dtype, pin_memory=True) for _ in range(num_layers)]
         self._ws = None
         self._ws_bytes = 0
+        self.prefill_out = None
 
     def close(self):
         self.sched.close()
@@ -140,6 +141,21 @@ class DecodeEngine:
             if len(idx.prompt_lens) else np.empty(0, np.int64)
         return reqs, pos
 
+    def prefill_indices(self, idx: StepIndices):
+        """Device index arrays of the step's prefill: the admitted prompts'
+        block tables (their rows of the step's tables), KV lengths (prompt
+        lengths: the decode token comes after), query_start over the new
+        positions prompt_starts .. prompt_lens - 1, and the longest run."""
+        dev = self.device
+        row = {int(r): i for i, r in enumerate(idx.running)}
+        rows = np.asarray([row[int(r)] for r in idx.prompt_seqs], np.int64)
+        counts = (idx.prompt_lens - idx.prompt_starts).astype(np.int64)
+        qs = np.zeros(len(rows) + 1, np.int32)
+        qs[1:] = np.cumsum(counts)
+        bt = torch.from_numpy(np.ascontiguousarray(idx.block_tables[rows])).to(dev)
+        sl = torch.from_numpy(idx.prompt_lens.astype(np.int32)).to(dev)
+        return bt, sl, torch.from_numpy(qs).to(dev), int(counts.max()) if len(counts) else 0
+
     # ---- device side -------------------------------------------------------------
     def workspace(self, batch):
         """A workspace large enough for `batch` sequences (grown on demand: the
@@ -175,7 +191,10 @@ class DecodeEngine:
 
         inputs: per layer l, a dict with "q" [n][H][D], "k_dec", "v_dec" [n][Hkv][D]
         (the new token of each running request) and "k_prompt", "v_prompt"
-        [T][Hkv][D] (the prompt K/V in prompt_slots order), all on the device.
+        [T][Hkv][D] (the prompt K/V in prompt_slots order), all on the device;
+        with "q_prompt" [T][H][D] (prompt queries, same order) the admitted
+        prompts' causal prefill attention runs too (pa_prefill, after the prompt
+        append), its outputs kept in self.prefill_out[l].
         Returns the attention outputs per layer ([n][H][D] each)."""
         dev = self.device
         n = len(idx.running)
@@ -189,6 +208,8 @@ class DecodeEngine:
         cd = torch.from_numpy(idx.cow_dst).to(dev) if len(idx.cow_dst) else None
         ws = self.workspace(n)
         self.run_swaps(idx)
+        pf = self.prefill_indices(idx) if (ps is not None and "q_prompt" in inputs[0]) else None
+        self.prefill_out = [] if pf is not None else None
         outs = out if out is not None else [torch.empty(n, self.num_heads, self.head_dim,
                                                          dtype=self.pools[0].dtype, device=dev)
                                              for _ in range(self.num_layers)]
@@ -198,6 +219,12 @@ class DecodeEngine:
                 bd.pa_copy_blocks(pool, cs, cd)
             if ps is not None:
                 bd.pa_reshape_and_cache(x["k_prompt"], x["v_prompt"], pool, ps)
+            if pf is not None:
+                # the admitted prompts' new positions attend causally over their KV
+                pbt, psl, pqs, pmax = pf
+                po = torch.empty_like(x["q_prompt"])
+                bd.pa_prefill(po, x["q_prompt"], pool, pbt, psl, pqs, self.scale, pmax)
+                self.prefill_out.append(po)
             # each running request's new token appended and attended in one call
             bd.pa_append_decode(outs[l], x["q"], x["k_dec"], x["v_dec"], pool, ds, bt, sl, self.scale,
                                 self.max_seq_len, ws)
@@ -207,7 +234,8 @@ class DecodeEngine:
 class GraphedLayers:
     """The decode part of a step over all layers (each running request's new
     token appended and attended: pa_append_decode per layer) replayed as one
-    CUDA graph per batch-size bucket.
+    CUDA graph per batch-size bucket (prompt appends, prefill attention and
+    copy-on-write copies, whose sizes vary every step, run eagerly first).
 
     Padded rows have length 0 and slot -1: they append nothing and their
     output rows are zeros, so a bucket's graph serves any batch up to its size.
@@ -276,11 +304,17 @@ class GraphedLayers:
         cs = torch.from_numpy(idx.cow_src).to(dev) if len(idx.cow_src) else None
         cd = torch.from_numpy(idx.cow_dst).to(dev) if len(idx.cow_dst) else None
         ps = torch.from_numpy(idx.prompt_slots).to(dev, non_blocking=True) if len(idx.prompt_slots) else None
+        pf = e.prefill_indices(idx) if (ps is not None and "q_prompt" in inputs[0]) else None
+        e.prefill_out = [] if pf is not None else None
         for l, pool in enumerate(e.pools):
             if cs is not None:
                 bd.pa_copy_blocks(pool, cs, cd)
             if ps is not None:
                 bd.pa_reshape_and_cache(inputs[l]["k_prompt"], inputs[l]["v_prompt"], pool, ps)
+            if pf is not None:
+                po = torch.empty_like(inputs[l]["q_prompt"])
+                bd.pa_prefill(po, inputs[l]["q_prompt"], pool, pf[0], pf[1], pf[2], e.scale, pf[3])
+                e.prefill_out.append(po)
         # static buffers: this step's rows, then inert padding up to the bucket
         self.bt[:n].copy_(torch.from_numpy(idx.block_tables), non_blocking=True)
         self.sl[:n].copy_(torch.from_numpy(idx.seq_lens), non_blocking=True)

@@ -113,7 +113,7 @@ TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
 
 # value-stream tags
 TAG_POOL, TAG_Q, TAG_K, TAG_V = 1, 2, 3, 4
-TAG_TRACE_KV, TAG_TRACE_Q = 5, 6
+TAG_TRACE_KV, TAG_TRACE_Q, TAG_TRACE_PQ = 5, 6, 7
 
 
 # ---------------------------------------------------------------------------
@@ -422,12 +422,24 @@ class TraceCase:
         x = x.reshape(len(r), 2, self.num_kv_heads, self.head_dim)
         return x[:, 0].contiguous(), x[:, 1].contiguous()
 
+    def prompt_q_values(self, layer: int, reqs, positions, device="cpu"):
+        """Query of prompt token `positions[i]` of request `reqs[i]` in `layer`
+        (the prefill queries): [n][H][D]. The same (layer, request, position)
+        always gives the same values."""
+        per = self.num_heads * self.head_dim
+        r = torch.as_tensor(np.asarray(reqs, dtype=np.int64), device=device)
+        p = torch.as_tensor(np.asarray(positions, dtype=np.int64), device=device)
+        c = ((r * TRACE_MAX_POS + p) * per)[:, None] + torch.arange(per, device=device)[None, :]
+        x = values(stream_key(self.seed, TAG_TRACE_PQ, layer), c).to(TORCH_DTYPE[self.dtype])
+        return x.reshape(len(r), self.num_heads, self.head_dim)
+
     def step_inputs(self, step: int, running, seq_lens, prompt_reqs, prompt_pos, device,
-                    chunk_elems: int = 1 << 26, stacked: bool = False):
+                    chunk_elems: int = 1 << 26, stacked: bool = False, prefill: bool = False):
         """Per-layer inputs of one continuous-batching step: the query and the
         new token's K/V of each running request (position seq_len - 1), and the
-        prompt K/V of the (re)admitted requests, generated layer by layer in
-        chunks of at most `chunk_elems` values."""
+        prompt K/V of the (re)admitted requests (with prefill, their prompt
+        queries too), generated layer by layer in chunks of at most
+        `chunk_elems` values."""
         per_tok = 2 * self.num_kv_heads * self.head_dim
         reqs_p = np.asarray(prompt_reqs, np.int64)
         pos_p = np.asarray(prompt_pos, np.int64)
@@ -462,7 +474,15 @@ class TraceCase:
                          for i in range(0, len(reqs_p), step_chunk)]
                 k_p = torch.cat([a for a, _ in parts])
                 v_p = torch.cat([b for _, b in parts])
-            out.append({"q": q, "k_dec": k_d, "v_dec": v_d, "k_prompt": k_p, "v_prompt": v_p})
+            item = {"q": q, "k_dec": k_d, "v_dec": v_d, "k_prompt": k_p, "v_prompt": v_p}
+            if prefill:
+                per_q_tok = self.num_heads * self.head_dim
+                qchunk = max(1, chunk_elems // per_q_tok)
+                item["q_prompt"] = torch.cat(
+                    [self.prompt_q_values(layer, reqs_p[i:i + qchunk], pos_p[i:i + qchunk], device)
+                     for i in range(0, len(reqs_p), qchunk)]) if len(reqs_p) else \
+                    torch.empty(0, self.num_heads, self.head_dim, dtype=dt, device=device)
+            out.append(item)
         if stacked:
             return out, (q_all, kv_all[:, :, 0], kv_all[:, :, 1])
         return out

@@ -176,3 +176,70 @@ def test_shared_prompt_trace_with_prefix_caching_matches_oracle():
     assert pk.pa_get_device_error() == 0
     assert cached_total > 0 and hits_checked >= 5 and checked >= 20, (cached_total, hits_checked, checked)
     eng.close()
+
+
+def oracle_prefill_row(trace, layer, req, table, length, pos):
+    """Oracle: the prompt token at `pos` of a request whose first `length`
+    positions hold the generator's K/V (written through its own table),
+    attending causally to positions 0..pos, in fp64."""
+    ids = sorted(set(table))
+    remap = {b: i for i, b in enumerate(ids)}
+    pool = np.zeros((len(ids), 2, trace.num_kv_heads, 16, trace.head_dim), dtype=np.uint16)
+    k, v = trace.kv_values(layer, [req] * length, np.arange(length), "cpu")
+    slots = [remap[table[p // 16]] * 16 + p % 16 for p in range(length)]
+    assert oa.reshape_and_cache(pool, storage_bits(k), storage_bits(v), slots) == []
+    q = storage_bits(trace.prompt_q_values(layer, [req], [pos], "cpu"))
+    tab = [[remap[b] for b in table]]
+    return oa.paged_prefill(q, pool, tab, [pos + 1], [1], trace.scale, "bf16")[0]
+
+
+def test_trace_with_prefill_attention_matches_oracle():
+    """The step loop with prefill attention on: each step's admitted prompts
+    (fresh and recomputed after preemption) attend causally over their paged KV
+    (pa_prefill after the prompt append). Sampled prompt rows match the fp64
+    oracle; decode outputs of the same steps are unaffected."""
+    from oracle_side import prefill_tolerance_ok
+    trace = wl.trace_case(seed=7, n_requests=120, rate=12.0, num_blocks=1200, num_layers=2,
+                          output_cap=200)
+    eng = DecodeEngine(trace.num_blocks, trace.num_layers, trace.num_heads, trace.num_kv_heads,
+                       trace.head_dim, trace.arrival_step, trace.prompt_len, trace.output_len,
+                       trace.table_width, trace.scale, DEV)
+    rng = np.random.default_rng(1)
+    checked = prompts_seen = 0
+    while True:
+        idx = eng.schedule()
+        if len(idx.running):
+            reqs_p, pos_p = eng.prompt_positions(idx)
+            inputs, _ = trace.step_inputs(idx.step, idx.running, idx.seq_lens, reqs_p, pos_p, DEV,
+                                          stacked=True, prefill=True)
+            eng.run_layers(idx, inputs)
+            if len(idx.prompt_seqs):
+                prompts_seen += len(idx.prompt_seqs)
+                assert eng.prefill_out is not None and len(eng.prefill_out) == trace.num_layers
+                assert pk_device_error() == 0
+                if checked < 24:
+                    layer = int(rng.integers(0, trace.num_layers))
+                    starts = np.concatenate([[0], np.cumsum(idx.prompt_lens - idx.prompt_starts)])
+                    row_of = {int(r): i for i, r in enumerate(idx.running)}
+                    got_all = eng.prefill_out[layer].float().cpu().numpy()
+                    for k in rng.choice(len(idx.prompt_seqs), size=min(2, len(idx.prompt_seqs)), replace=False):
+                        req = int(idx.prompt_seqs[k])
+                        n_new = int(idx.prompt_lens[k] - idx.prompt_starts[k])
+                        for i in {0, n_new - 1, int(rng.integers(n_new))}:
+                            pos = int(idx.prompt_starts[k]) + i
+                            table = idx.block_tables[row_of[req]].tolist()
+                            ref = oracle_prefill_row(trace, layer, req, table, int(idx.prompt_lens[k]), pos)
+                            ok, err, _ = prefill_tolerance_ok(got_all[int(starts[k]) + i], ref)
+                            assert ok, (idx.step, req, pos, err)
+                            checked += 1
+            else:
+                assert eng.prefill_out is None
+        if idx.done:
+            break
+    eng.close()
+    assert checked >= 24 and prompts_seen >= 100
+
+
+def pk_device_error():
+    import paged_kv_cache_400_b200 as pk
+    return pk.pa_get_device_error()
