@@ -439,6 +439,7 @@ def run_ours(args, rank, world, dist):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": cfg,
+        "tokens_per_s_32_layer_equiv": value / 32,
         "kv_read_gbs": kv_gbs, "kv_frac_of_8tbs": kv_gbs / NOMINAL_HBM_GBS,
         "kv_frac_of_measured": kv_gbs / peak,
         "roofline": {"kernel": "decode_staged_kernel with fused append (pa_append_decode; partition "
