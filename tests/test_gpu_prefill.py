@@ -151,6 +151,36 @@ def test_chunked_prefill_full_size_sampled():
     _sampled(wl.chunked_prefill_case(0), 24, 1)
 
 
+def test_long_context_chunk():
+    # a 96-token chunk after 30 000 cached tokens (1882 blocks): long KV loops,
+    # block ids read in many batches, a wide table
+    case = wl.prefill_custom("long_ctx", 9, [30000, 200], [96, 40], 32, 8)
+    prep = prepare_prefill_step(case)
+    ost = oracle_prefill_indices(case)
+    check_indices(case, prep, ost)
+    pool, out = device_prefill(case, prep)
+    assert pk.pa_get_device_error() == 0
+    picks = [(0, 0), (0, 31), (0, 32), (0, 95), (1, 0), (1, 39)]
+    ref = oracle_prefill_rows(case, ost, picks)
+    got = np.stack([out[int(prep.query_start[b]) + i].float().cpu().numpy() for b, i in picks])
+    ok, err, _ = prefill_tolerance_ok(got, ref)
+    assert ok, err
+
+
+def test_mha_full_prompts_sampled():
+    # G = 1: 128 tokens per query tile, whole prompts up to 1000 tokens
+    case = wl.prefill_custom("mha_prompts", 10, [0, 0, 0, 0], [1000, 129, 128, 5], 32, 32)
+    prep = prepare_prefill_step(case)
+    ost = oracle_prefill_indices(case)
+    pool, out = device_prefill(case, prep)
+    assert pk.pa_get_device_error() == 0
+    picks = [(0, 0), (0, 127), (0, 128), (0, 255), (0, 999), (1, 128), (2, 127), (3, 4)]
+    ref = oracle_prefill_rows(case, ost, picks)
+    got = np.stack([out[int(prep.query_start[b]) + i].float().cpu().numpy() for b, i in picks])
+    ok, err, _ = prefill_tolerance_ok(got, ref)
+    assert ok, err
+
+
 def test_last_row_matches_decode():
     # the newest token's prefill row attends to the whole sequence, as decode does
     case = wl.prefill_custom("vs_decode", 6, [100, 0, 31], [50, 77, 1], 32, 8)
