@@ -69,7 +69,7 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
 }
 
 // 5-D tiled TMA load of one box into shared memory, completion signalled on
-// `bar` as transaction bytes. No multicast.
+// `bar` as transaction bytes; the box lands in this CTA's shared memory only.
 __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t c0,
                                             int32_t c1, int32_t c2, int32_t c3, int32_t c4) {
   asm volatile(
