@@ -34,3 +34,54 @@ def test_row_sampling_matches_whole_step():
     picks = [(b, i) for b in range(3) for i in range(case.query_lens[b])]
     rows = oracle_prefill_rows(case, ost, picks)
     assert np.allclose(rows, whole, rtol=0, atol=1e-12)
+
+
+def test_prefill_flop_count_closed_form():
+    """The prefill roofline's algorithmic FLOPs: for every new position p of a
+    sequence, each query head scores p + 1 keys and sums p + 1 values, 2 x 128
+    FLOPs each. The bench's closed form against a brute-force count."""
+    import bench
+    case = wl.prefill_custom("f", 3, [0, 7, 100, 16], [5, 1, 33, 0], 32, 8)
+    brute = 0
+    for c, n in zip(case.ctx_lens, case.query_lens):
+        for p in range(c, c + n):
+            brute += case.num_heads * (p + 1) * 2 * 2 * case.head_dim
+    assert bench.prefill_flops(case) == brute
+
+
+def test_engine_prefill_indices_match_oracle_replay():
+    """DecodeEngine.prefill_indices (host side of the step loop's prefill):
+    per admitted prompt, its rows of the step's block tables, KV length =
+    prompt length, and query_start over the new positions, against the
+    oracle scheduler's replay of the same trace (CPU)."""
+    import torch
+    from oracle.block_manager import OracleBlockManager
+    from oracle.scheduler import OracleScheduler
+    from paged_kv_cache_400_b200.engine import DecodeEngine
+    trace = wl.trace_case(seed=3, n_requests=60, rate=8.0, num_blocks=400, num_layers=1, output_cap=80)
+    eng = DecodeEngine(trace.num_blocks, 1, 4, 2, 128, trace.arrival_step, trace.prompt_len,
+                       trace.output_len, trace.table_width, trace.scale, "cpu")
+    obm = OracleBlockManager(trace.num_blocks)
+    osch = OracleScheduler(obm, trace.arrival_step, trace.prompt_len, trace.output_len, trace.table_width)
+    seen = 0
+    while True:
+        idx = eng.schedule()
+        o = osch.step()
+        if len(idx.prompt_seqs):
+            bt, sl, qs, mx = eng.prefill_indices(idx)
+            bt, sl, qs = bt.numpy(), sl.numpy(), qs.numpy()
+            running = o["running"]
+            starts = o.get("prompt_starts", [0] * len(o["prompt_seqs"]))
+            for k, req in enumerate(o["prompt_seqs"]):
+                row = running.index(req)
+                assert sl[k] == o["prompt_lens"][k]
+                n_new = o["prompt_lens"][k] - starts[k]
+                assert qs[k + 1] - qs[k] == n_new
+                width = (o["prompt_lens"][k] + 15) // 16
+                assert bt[k, :width].tolist() == o["block_tables"][row][:width]
+            assert qs[0] == 0 and mx == max(int(a) - int(b) for a, b in zip(o["prompt_lens"], starts))
+            seen += len(o["prompt_seqs"])
+        if idx.done:
+            break
+    eng.close()
+    assert seen >= 60
