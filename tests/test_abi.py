@@ -68,6 +68,34 @@ def test_decode_rejects_bad_arguments_on_host():
     assert L.pa_decode(None, None, None, None, 4, None, 0, 2, 0.1, p, None, 0, 16, None) == 0
 
 
+def test_prefill_rejects_bad_arguments_on_host():
+    L = bd.lib()
+    vp = C.c_void_p(16)  # never dereferenced: rejected before use
+    p = pool(heads=8)
+    # (out, q, pool, tables, max_blocks, seq_lens, query_start, num_seqs, num_tokens, H, scale, desc, max_q)
+    ok_args = (vp, vp, vp, vp, 4, vp, vp, 2, 64, 32, 0.1, p, 40, None)
+    def call(**kw):
+        a = list(ok_args)
+        names = ["out", "q", "kv", "bt", "mb", "sl", "qs", "ns", "nt", "H", "scale", "desc", "mq", "st"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return L.pa_prefill(*a)
+    assert call(desc=pool(heads=8, dtype=bd.PA_F32)) == 2     # only bf16
+    assert call(desc=pool(heads=8, dim=64)) == 2              # only head_dim 128
+    assert call(H=24) == 2                                    # group of 3: not a power of two
+    assert call(H=36) == 1                                    # H not a multiple of Hkv
+    assert call(H=256) == 2                                   # group of 32
+    assert call(mq=65) == 1                                   # longer than the tokens given
+    assert call(mq=80, nt=100) == 1                           # beyond max_blocks * 16
+    assert call(scale=float("inf")) == 1
+    assert call(q=None) == 1
+    assert call(out=C.c_void_p(24)) == 1                      # misaligned
+    assert call(ns=-1) == 1
+    assert call(ns=0) == 0                                    # nothing to do
+    assert call(mq=0, nt=0) == 0
+    assert call(desc=pool(heads=8, bs=32)) == 2               # block size must be 16
+
+
 def test_append_and_copy_reject_bad_arguments_on_host():
     L = bd.lib()
     vp = C.c_void_p(16)
