@@ -181,6 +181,39 @@ def test_mha_full_prompts_sampled():
     assert ok, err
 
 
+def test_physical_permutation_is_bit_invariant():
+    # relabelling every physical block (pool rows moved, tables rewritten) must
+    # not change a single output bit: placement never enters the arithmetic
+    case = wl.prefill_custom("perm", 11, [0, 45, 300], [90, 64, 33], 32, 8)
+    prep = prepare_prefill_step(case)
+    pool, out = device_prefill(case, prep)
+    perm = torch.from_numpy(np.random.default_rng(3).permutation(case.num_blocks)).to(DEV)
+    pool2 = torch.empty_like(pool)
+    pool2[perm] = pool
+    bt = torch.from_numpy(prep.block_tables).to(DEV).long()
+    bt2 = torch.where(bt >= 0, perm[bt.clamp(min=0)], bt).int()
+    out2 = torch.zeros_like(out)
+    pk.pa_prefill(out2, case.make_q(DEV), pool2, bt2.contiguous(), torch.from_numpy(prep.seq_lens).to(DEV),
+                  torch.from_numpy(prep.query_start).to(DEV), case.scale, case.max_query_len)
+    torch.cuda.synchronize()
+    assert pk.pa_get_device_error() == 0
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+
+
+def test_repeated_calls_are_deterministic():
+    case = wl.prefill_custom("det", 12, [10, 500], [200, 77], 32, 8)
+    prep = prepare_prefill_step(case)
+    pool, out = device_prefill(case, prep)
+    args = (case.make_q(DEV), pool, torch.from_numpy(prep.block_tables).to(DEV),
+            torch.from_numpy(prep.seq_lens).to(DEV), torch.from_numpy(prep.query_start).to(DEV),
+            case.scale, case.max_query_len)
+    for _ in range(3):
+        again = torch.zeros_like(out)
+        pk.pa_prefill(again, *args)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), again.view(torch.int16))
+
+
 def test_last_row_matches_decode():
     # the newest token's prefill row attends to the whole sequence, as decode does
     case = wl.prefill_custom("vs_decode", 6, [100, 0, 31], [50, 77, 1], 32, 8)
