@@ -413,3 +413,31 @@ def test_prefill_last_row_is_decode_and_first_token_sees_itself():
     assert np.array_equal(pre[-1], dec[0])
     for h in range(4):
         assert np.array_equal(pre[0, h], V[0][0, h // 2])
+
+
+def test_prefill_brute_force_fsum_tiny():
+    """Prefill oracle against sums written out with math.fsum: each new token at
+    position p scores positions 0..p only, softmax-normalised, over its own KV
+    head; chunks after cached context and GQA grouping included."""
+    rng = np.random.default_rng(31)
+    lens, qlens, n_heads, n_kv, d, scale = [9, 20], [9, 4], 4, 2, 4, 0.7
+    K, V = random_logical(rng, lens, n_kv, d)
+    pool, tables = scatter_logical(K, V, 8, rng)
+    q = rng.standard_normal((sum(qlens), n_heads, d))
+    out = oa.paged_prefill(q, pool, tables, lens, qlens, scale, "f64")
+    G = n_heads // n_kv
+    row = 0
+    for b, (L, n) in enumerate(zip(lens, qlens)):
+        for i in range(n):
+            p = L - n + i
+            for h in range(n_heads):
+                g = h // G
+                s = [scale * math.fsum(float(q[row + i, h, c]) * float(K[b][t, g, c]) for c in range(d))
+                     for t in range(p + 1)]
+                m = max(s)
+                e = [math.exp(x - m) for x in s]
+                z = math.fsum(e)
+                for c in range(d):
+                    o = math.fsum(e[t] * float(V[b][t, g, c]) for t in range(p + 1)) / z
+                    assert abs(out[row + i, h, c] - o) <= 1e-12 * max(1.0, abs(o))
+        row += n
