@@ -243,3 +243,47 @@ def test_trace_with_prefill_attention_matches_oracle():
 def pk_device_error():
     import paged_kv_cache_400_b200 as pk
     return pk.pa_get_device_error()
+
+
+def test_prefix_cached_prompts_prefill_matches_oracle():
+    """Prefill attention with prefix caching: a request whose system prompt
+    blocks are cached prefills only its positions from prompt_starts on, yet
+    those rows attend over the whole prompt, cached prefix included (written
+    by an earlier request). Sampled rows of cache-hit prompts vs the oracle."""
+    from oracle_side import prefill_tolerance_ok
+    trace = wl.prefix_trace_case(seed=9, n_requests=90, rate=10.0, num_blocks=2400, num_layers=2, n_system=2)
+    trace.output_len = np.minimum(trace.output_len, 120).astype(np.int32)
+    eng = DecodeEngine(trace.num_blocks, trace.num_layers, trace.num_heads, trace.num_kv_heads,
+                       trace.head_dim, trace.arrival_step, trace.prompt_len, trace.output_len,
+                       trace.table_width, trace.scale, DEV, prompt_tokens=trace.prompt_tokens)
+    rng = np.random.default_rng(4)
+    hits = checked = 0
+    while True:
+        idx = eng.schedule()
+        if len(idx.running):
+            reqs_p, pos_p = eng.prompt_positions(idx)
+            inputs, _ = trace.step_inputs(idx.step, idx.running, idx.seq_lens, reqs_p, pos_p, DEV,
+                                          stacked=True, prefill=True)
+            eng.run_layers(idx, inputs)
+            cached = [k for k in range(len(idx.prompt_seqs)) if idx.prompt_starts[k] > 0]
+            if cached and checked < 24:
+                layer = int(rng.integers(0, trace.num_layers))
+                starts = np.concatenate([[0], np.cumsum(idx.prompt_lens - idx.prompt_starts)])
+                row_of = {int(r): i for i, r in enumerate(idx.running)}
+                got_all = eng.prefill_out[layer].float().cpu().numpy()
+                for k in cached[:2]:
+                    req = int(idx.prompt_seqs[k])
+                    n_new = int(idx.prompt_lens[k] - idx.prompt_starts[k])
+                    table = idx.block_tables[row_of[req]].tolist()
+                    for i in {0, n_new - 1, int(rng.integers(n_new))}:
+                        pos = int(idx.prompt_starts[k]) + i
+                        ref = oracle_prefill_row(trace, layer, req, table, int(idx.prompt_lens[k]), pos)
+                        ok, err, _ = prefill_tolerance_ok(got_all[int(starts[k]) + i], ref)
+                        assert ok, (idx.step, req, pos, err)
+                        checked += 1
+                    hits += 1
+        if idx.done:
+            break
+    eng.close()
+    assert pk_device_error() == 0
+    assert hits >= 5 and checked >= 15
