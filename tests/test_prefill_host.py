@@ -85,3 +85,39 @@ def test_engine_prefill_indices_match_oracle_replay():
             break
     eng.close()
     assert seen >= 60
+
+
+def test_prefill_indices_skip_swapped_in_requests():
+    """Swap-mode preemption: a request swapped back in has its KV restored by
+    block copies, so it is not among the step's prompts and gets no prefill
+    rows; every prompt that is prefilled is fresh or recomputed (CPU, through
+    the library's scheduler)."""
+    from types import SimpleNamespace
+
+    import torch
+    from paged_kv_cache_400_b200 import binding as bd
+    from paged_kv_cache_400_b200.engine import DecodeEngine
+    trace = wl.trace_case(seed=5, n_requests=240, rate=16.0, num_blocks=1800, num_layers=1, output_cap=300)
+    bm = bd.BlockManager(trace.num_blocks)
+    sched = bd.Scheduler(bm, trace.arrival_step, trace.prompt_len, trace.output_len, trace.table_width)
+    sched.set_swap(600)
+    # DecodeEngine's host-side methods on a stand-in engine (no device pools)
+    eng = SimpleNamespace(sched=sched, device=torch.device("cpu"))
+    swapped_in_total = prompts_total = 0
+    while True:
+        idx = DecodeEngine.schedule(eng)
+        swapped = {int(d) for d in idx.swap_in[:, 1]} if len(idx.swap_in) else set()
+        if len(idx.prompt_seqs):
+            bt, sl, qs, mx = DecodeEngine.prefill_indices(eng, idx)
+            prompts_total += len(idx.prompt_seqs)
+            assert (np.diff(qs.numpy()) == idx.prompt_lens - idx.prompt_starts).all()
+            # no prefilled prompt's table holds a block the step swaps in
+            width = (idx.prompt_lens + 15) // 16
+            for k in range(len(idx.prompt_seqs)):
+                assert not (set(bt.numpy()[k, :width[k]].tolist()) & swapped)
+        swapped_in_total += len(idx.swap_in)
+        if idx.done:
+            break
+    sched.close()
+    bm.close()
+    assert prompts_total > 200 and swapped_in_total > 0
