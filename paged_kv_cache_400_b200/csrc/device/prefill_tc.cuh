@@ -133,7 +133,10 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
   const int32_t nt_max = (nblocks + kTcBlocksPerTile - 1) / kTcBlocksPerTile;
   const int32_t* table = p.block_tables + (size_t)b * p.max_blocks;
 
-  if (threadIdx.x == 0) {
+  // The producer warp sets up the mbarriers and starts loading at once; the
+  // other warps wait on named barrier 1 (which the producer only arrives at)
+  // and the MMA warp allocates tensor memory meanwhile.
+  if (warp == Cfg::kProducerWarp && lane == 0) {
     mbar_init(&sh.q_full, 1);
 #pragma unroll
     for (int s = 0; s < S; ++s) {
@@ -156,10 +159,15 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
     tmem_alloc(&sh.tmem_base, Cfg::kTmemCols);
     tmem_relinquish();
   }
-  tc_fence_before_sync();
-  __syncthreads();
-  tc_fence_after_sync();
-  const uint32_t tmem = sh.tmem_base;
+  if (warp == Cfg::kProducerWarp) {
+    __syncwarp();
+    named_barrier_arrive(1, Cfg::kThreads);
+  } else {
+    tc_fence_before_sync();
+    named_barrier_sync(1, Cfg::kThreads);
+    tc_fence_after_sync();
+  }
+  const uint32_t tmem = sh.tmem_base;  // read by the MMA and softmax warps only
 
   if (warp == Cfg::kProducerWarp) {
     // ---- producer ---------------------------------------------------------------
