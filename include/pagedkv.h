@@ -244,6 +244,11 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* kv_pool,
  * from it). A wait on staged data that exceeds 2 s sets PA_DEVERR_TIMEOUT; while
  * that bit is set (until pa_get_device_error reads it), prefill tiles that
  * start later skip their work. Allocates nothing.
+ * Kernel: tcgen05 MMAs with tensor-memory accumulators, two 128-row query
+ * tiles per CTA. For comparison only, the environment variable
+ * PAGEDKV_PREFILL_KERNEL=mma_sync selects an mma.sync kernel and
+ * PAGEDKV_PREFILL_QTILES=1 a one-tile tcgen05 variant (same results within
+ * rounding; read at every call).
  */
 pa_status pa_prefill(void* out, const void* q, const void* kv_pool,
                      const int32_t* block_tables, int32_t max_blocks_per_seq,
