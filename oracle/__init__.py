@@ -12,8 +12,8 @@ Modules
                  and block copy.
   block_manager  integer block manager: FIFO free list, page tables, refcounts,
                  fork, copy-on-write of a shared partial last block, free.
-  scheduler      integer continuous-batching step loop with recompute
-                 preemption.
+  scheduler      integer continuous-batching step loop with recompute and
+                 swap-mode preemption.
 
 Sources: three web pages on PagedAttention —
   "大模型推理性能优化：PagedAttention与Continuous Batching原理与实践",
@@ -22,7 +22,8 @@ Sources: three web pages on PagedAttention —
 Each function names the page section it follows.
 
 Parity status: every function here is pinned by tests/test_oracle_pins.py and
-tests/test_oracle_scheduler.py; the scheduler's step-order details beyond the
-pinned policy points are "parity unpinned" (checked by invariants and by
-hand-written event lists on tiny traces only).
+tests/test_oracle_scheduler.py (swap mode included: hand-worked event lists for
+each swap rule and a host-block accounting invariant on a random trace); the
+scheduler's step-order details beyond the pinned policy points are checked by
+invariants and by hand-written event lists on tiny traces only.
 """

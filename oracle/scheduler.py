@@ -9,8 +9,8 @@ Sources:
       allocating their pages, 3) runs one forward step over the running set,
       4) appends each request's new token to its KV cache.
       "Preemption（抢占）": when memory runs short a lower-priority request is
-      suspended, its pages freed, and it resumes later by recomputation (or
-      swap; only recompute is modelled here).
+      suspended, its pages freed, and it resumes later by recomputation or,
+      in swap mode, from a copy of its KV in CPU memory.
       "Continuous Batching": requests join as they arrive and leave as soon as
       they finish.
   "大模型推理性能优化：PagedAttention与Continuous Batching原理与实践" §2.3: a global
