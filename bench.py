@@ -58,6 +58,8 @@ def parse_args():
                     help="prefix_trace: run without automatic prefix caching (for comparison)")
     ap.add_argument("--prefill", action="store_true",
                     help="trace: also run the admitted prompts' causal prefill attention (pa_prefill) per layer")
+    ap.add_argument("--prefill-kernel", choices=["tcgen05", "tcgen05_1tile", "mma_sync"], default="tcgen05",
+                    help="prefill workloads: the product kernel, or a comparison build's kernel")
     ap.add_argument("--graphs", action="store_true",
                     help="trace: replay each step's decode over all layers as a CUDA graph")
     ap.add_argument("--batch", type=int, default=256,
@@ -807,7 +809,7 @@ def run_prefill(args, rank, world, dist):
     if rank != 0:
         return
     flops = prefill_flops(case)
-    mma_sync = os.environ.get("PAGEDKV_PREFILL_KERNEL") == "mma_sync"
+    mma_sync = args.prefill_kernel == "mma_sync"
     att_avg = sum(att_ms) / K
     peak, peak_src = measured_tensor_peak()
     achieved = flops / (att_avg / 1e3) / 1e12
@@ -815,7 +817,7 @@ def run_prefill(args, rank, world, dist):
         case.num_kv_heads * case.head_dim * 2
     traffic, traffic_src = None, ("mma.sync kernel: not captured" if mma_sync else
                                   "captured at 64 sequences only")
-    if not mma_sync and pb == 64:
+    if args.prefill_kernel == "tcgen05" and pb == 64:
         traffic, traffic_src = recorded_traffic(
             os.path.join(ROOT, "profiles", f"prefill_tc_{'chunked' if chunked else 'prompts'}_b64.md"),
             PREFILL_KERNEL_SOURCES)
@@ -833,8 +835,10 @@ def run_prefill(args, rank, world, dist):
                    "parallelism": f"dp{world} independent replicas (no exchange step)",
                    "l2": "no flush: K/V read %.2f GB per step (> 126 MB L2), q/out %.2f GB"
                          % (kv_bytes / 1e9, 2 * T * case.num_heads * case.head_dim * 2 / 1e9)},
-        "roofline": {"kernel": ("prefill_kernel (mma.sync m16n8k16)" if mma_sync else
-                                "prefill_tc_kernel (tcgen05.mma, accumulators in tensor memory)"),
+        "roofline": {"kernel": ("prefill_kernel (mma.sync m16n8k16; comparison build)" if mma_sync else
+                                "prefill_tc_kernel (tcgen05.mma, accumulators in tensor memory)"
+                                + ("; one query tile per CTA, comparison build"
+                                   if args.prefill_kernel == "tcgen05_1tile" else "")),
                      "bound": "tensor", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_src,
                      "traffic": traffic, "traffic_source": traffic_src,
@@ -882,7 +886,11 @@ def main():
         elif args.workload in ("trace", "prefix_trace"):
             run_trace(args, rank, world)
         elif args.workload in ("prefill", "chunked_prefill"):
-            run_prefill(args, rank, world, dist)
+            from paged_kv_cache_400_b200 import binding as bd
+            variant = {"tcgen05": None, "tcgen05_1tile": "prefill_1tile",
+                       "mma_sync": "prefill_mma_sync"}[args.prefill_kernel]
+            with bd.use_variant(variant):
+                run_prefill(args, rank, world, dist)
         else:
             run_ours(args, rank, world, dist)
     finally:

@@ -111,15 +111,19 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, void* kv_pool,
 /*
  * Bytes of device workspace pa_decode needs for this shape (split-KV partial
  * results). 0 means pa_decode needs none and accepts workspace == NULL.
- * Depends only on the arguments. Returns 0 for invalid arguments too, which
- * pa_decode then rejects.
+ * Depends on the arguments and on the current device's SM count (read once per
+ * device; 148, a B200's, when no device can be queried), so size the
+ * workspace with the device current that pa_decode will run on. Returns 0 for
+ * invalid arguments too, which pa_decode then rejects.
  */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads,
                                 pa_pool_desc pool, int32_t max_seq_len);
 
 /*
- * Tokens per split-KV partition that pa_decode uses for this shape (a
- * multiple of 16). Sequences no longer than this are finished in one pass.
+ * Tokens per split-KV partition that pa_decode uses for this shape on the
+ * current device (a multiple of 16): 2048, halved down to 128 while the
+ * (sequence, KV head, partition) grid would give the device's SMs fewer than
+ * four CTAs each. Sequences no longer than this are finished in one pass.
  */
 int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_heads,
                                    pa_pool_desc pool, int32_t max_seq_len);
@@ -199,9 +203,12 @@ pa_status pa_append_decode(void* out, const void* q, const void* k_new, const vo
  * Same arguments, results and errors as pa_decode, minus the workspace. This
  * call allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *  - The first call on a device looks up the array's device address (once per
- *    device, with that device current); make that first call before any
- *    stream capture.
- *  - A shape whose partial results need more than
+ *    device, with that device current) and keeps it for the life of the
+ *    process; make that first call before any stream capture. cudaDeviceReset
+ *    on that device ends the context the address belongs to: calling this
+ *    entry point after a reset is not supported.
+ *  - Arguments are checked exactly as pa_decode checks them, and those errors
+ *    come first; then a shape whose partial results need more than
  *    PA_DECODE_NOALLOC_SCRATCH_BYTES (pa_decode_workspace_size) is rejected
  *    with PA_ERR_WORKSPACE before anything is enqueued; use pa_decode then.
  *  - Every call uses the same array and it keeps the last call's contents.
@@ -245,10 +252,10 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* kv_pool,
  * that bit is set (until pa_get_device_error reads it), prefill tiles that
  * start later skip their work. Allocates nothing.
  * Kernel: tcgen05 MMAs with tensor-memory accumulators, two 128-row query
- * tiles per CTA. For comparison only, the environment variable
- * PAGEDKV_PREFILL_KERNEL=mma_sync selects an mma.sync kernel and
- * PAGEDKV_PREFILL_QTILES=1 a one-tile tcgen05 variant (same results within
- * rounding; read at every call).
+ * tiles per CTA. There is no run-time kernel choice: the mma.sync kernel and a
+ * one-tile tcgen05 variant exist only in separate comparison builds of this
+ * library (compiled with PA_PREFILL_MMA_SYNC or PA_PREFILL_QTILES=1; same
+ * results within rounding).
  */
 pa_status pa_prefill(void* out, const void* q, const void* kv_pool,
                      const int32_t* block_tables, int32_t max_blocks_per_seq,

@@ -8,6 +8,7 @@ If the library cannot be loaded (not built, nvcc missing) every call raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes as C
 import os
 import threading
@@ -106,6 +107,7 @@ def _declare(lib):
         "pa_bm_evictable_list": (i32, [vp, _P32, i32, _P32]),
         "pa_bm_num_cached": (i32, [vp]),
         "pa_prefill": (i32, [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, f32, pa_pool_desc, i32, vp]),
+        "pa_decode_noalloc": (i32, [vp, vp, vp, vp, i32, vp, i32, i32, f32, pa_pool_desc, i32, vp]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -114,9 +116,16 @@ def _declare(lib):
     return lib
 
 
+_variant = None       # name of the comparison build in use, None for the product library
+_variant_libs = {}
+
+
 def lib():
-    """The loaded library (built first if missing or stale)."""
+    """The loaded library (built first if missing or stale): the product
+    library, or the comparison build selected by use_variant()."""
     global _lib
+    if _variant is not None:
+        return _variant_libs[_variant]
     if _lib is None:
         with _lock:
             if _lib is None:
@@ -125,8 +134,27 @@ def lib():
     return _lib
 
 
+@contextlib.contextmanager
+def use_variant(name):
+    """Routes every call of this module to a comparison build of the library
+    (build.VARIANTS, e.g. "prefill_mma_sync") until the block exits; None keeps
+    the product library. For comparisons and their tests only; not
+    thread-safe."""
+    global _variant
+    if name is not None and name not in _variant_libs:
+        with _lock:
+            if name not in _variant_libs:
+                _variant_libs[name] = _declare(C.CDLL(_build.build(variant=name)))
+    prev = _variant
+    _variant = name
+    try:
+        yield
+    finally:
+        _variant = prev
+
+
 def library_path() -> str:
-    return _build.LIB
+    return _build.lib_path(_variant)
 
 
 def _check(fn: str, status: int):
@@ -263,9 +291,6 @@ def pa_decode_noalloc(out, q, kv_pool, block_tables, seq_lens, scale, max_seq_le
     (PagedKVError WORKSPACE). Calls overlapping on the GPU share that array and
     race."""
     fn = lib().pa_decode_noalloc
-    fn.restype = C.c_int32
-    fn.argtypes = [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_int32,
-                   C.c_int32, C.c_float, pa_pool_desc, C.c_int32, C.c_void_p]
     desc = pool_desc(kv_pool)
     B, H, D = q.shape
     if out.shape != q.shape or D != desc.head_dim:

@@ -4,6 +4,12 @@ One shared library: the CUDA translation unit (all kernels + device C-ABI
 entry points) and the host C++ block manager / scheduler. CUDA runtime is
 linked statically; only the pa_* symbols are exported. A digest of the sources
 and flags is stored beside the library; build() rebuilds only when it changes.
+
+Comparison builds (build(variant=...)) compile the same sources with one
+compile-time switch into a library of their own, libpagedkv_<variant>.so; the
+product library never contains their kernels:
+  prefill_mma_sync   pa_prefill runs the mma.sync prefill kernel
+  prefill_1tile      pa_prefill's tcgen05 kernel takes one query tile per CTA
 """
 from __future__ import annotations
 
@@ -25,6 +31,10 @@ SOURCES = [
     os.path.join(CSRC, "host", "block_manager.cpp"),
     os.path.join(CSRC, "host", "scheduler.cpp"),
 ]
+VARIANTS = {
+    "prefill_mma_sync": ["-DPA_PREFILL_MMA_SYNC"],
+    "prefill_1tile": ["-DPA_PREFILL_QTILES=1"],
+}
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
          "--expt-relaxed-constexpr", "-Xptxas", "-warn-spills"]
@@ -50,33 +60,47 @@ def _digest(extra) -> str:
     return h.hexdigest()
 
 
-def command(extra=()) -> list:
+def lib_path(variant=None) -> str:
+    """The product library, or a comparison build's library."""
+    if variant is None:
+        return LIB
+    if variant not in VARIANTS:
+        raise ValueError(f"unknown build variant {variant!r} (one of {sorted(VARIANTS)})")
+    return os.path.join(PKG, f"libpagedkv_{variant}.so")
+
+
+def command(extra=(), out=LIB) -> list:
     return ([nvcc_path()] + ARCH + FLAGS + list(extra) + ["-I", INCLUDE,
             "-Xlinker", "--version-script=" + os.path.join(CSRC, "exports.map"),
-            "-o", LIB] + SOURCES)
+            "-o", out] + SOURCES)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    digest = _digest(extra)
-    if not force and os.path.exists(LIB) and os.path.exists(STAMP):
-        with open(STAMP) as f:
+def build(force: bool = False, verbose: bool = False, extra=(), variant=None) -> str:
+    out = lib_path(variant)
+    flags = list(extra) + (VARIANTS[variant] if variant else [])
+    stamp = out + ".digest"
+    digest = _digest(flags)
+    if not force and os.path.exists(out) and os.path.exists(stamp):
+        with open(stamp) as f:
             if f.read().strip() == digest:
-                return LIB
-    cmd = command(extra)
+                return out
+    cmd = command(flags, out)
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
-    tmp = LIB + ".tmp"
+    tmp = out + ".tmp"
     cmd[cmd.index("-o") + 1] = tmp
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
-        raise RuntimeError("nvcc failed building libpagedkv.so:\n" + r.stdout + r.stderr)
+        raise RuntimeError(f"nvcc failed building {os.path.basename(out)}:\n" + r.stdout + r.stderr)
     if verbose and (r.stdout or r.stderr):
         print(r.stdout + r.stderr, file=sys.stderr)
-    os.replace(tmp, LIB)
-    with open(STAMP, "w") as f:
+    os.replace(tmp, out)
+    with open(stamp, "w") as f:
         f.write(digest + "\n")
-    return LIB
+    return out
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    names = [a[len("--variant="):] for a in sys.argv[1:] if a.startswith("--variant=")]
+    for v in (names or [None]):
+        print(build(force="--force" in sys.argv, verbose=True, variant=v))

@@ -41,7 +41,10 @@
 // their V rows are zeroed in shared memory first (unused pool rows may hold
 // any bits). A block id outside the pool is never loaded: the stage is marked
 // invalid (K and V read as zero) and PA_DEVERR_BLOCK is raised. Every mbarrier
-// wait gives up after 2 s and raises PA_DEVERR_TIMEOUT instead of hanging.
+// wait gives up after 2 s and raises PA_DEVERR_TIMEOUT instead of hanging; the
+// warp then issues no further copy, waits (bounded) for the ones it has in
+// flight, leaves its state out of the merge, and a persistent CTA takes no
+// further item.
 #pragma once
 
 #include <cudaTypedefs.h>
@@ -73,6 +76,7 @@ struct StagedShared {
   float red_m[kStagedWarps][16];
   float red_l[kStagedWarps][16];
   int32_t next_item;
+  int32_t abort;  // a warp of this CTA gave up on a stage: take no further items
 };
 
 // Attention over partition `part` of sequence b for KV head g (all G query
@@ -193,8 +197,31 @@ __device__ __forceinline__ void decode_partition(const CUtensorMap& tmap, const 
 
   for (int32_t i = 0; i < my; ++i) {
     const int32_t s = i % kStagedStages;
-    if (!mbar_wait_bounded(&bars[warp][s], (phase >> s) & 1u, kWaitLimitNs)) {
+    const bool arrived = mbar_wait_bounded(&bars[warp][s], (phase >> s) & 1u, kWaitLimitNs);
+    if (__any_sync(0xffffffffu, !arrived)) {
+      // Gave up on this stage: raise PA_DEVERR_TIMEOUT, issue nothing more,
+      // wait (bounded) for the copies already issued into this warp's stages
+      // (blocks i .. min(i + stages, my) - 1) so none lands after the CTA
+      // leaves, and drop this warp's state from the merge. The sequence's
+      // output is then undefined; the error word says so.
       if (lane == 0) raise_device_error(PA_DEVERR_TIMEOUT);
+      const int32_t issued = min(i + kStagedStages, my);
+      for (int32_t k = i; k < issued; ++k) {
+        const int32_t sk = k % kStagedStages;
+        mbar_wait_bounded(&bars[warp][sk], (phase >> sk) & 1u, kWaitLimitNs);
+        phase ^= 1u << sk;
+      }
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+      if constexpr (kMMA) {
+#pragma unroll
+        for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+      }
+      if (lane == 0) sh.abort = 1;
+      break;
     }
     phase ^= 1u << s;
     const int32_t tok0 = t0 + (warp + i * kStagedWarps) * 16;
@@ -460,10 +487,13 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constan
   }
   grid_dependency_wait();  // the plan kernel's item list is complete
   const int32_t total = __ldcg(p.work_header) * p.num_kv_heads;
-  if (threadIdx.x == 0) sh.next_item = atomicAdd(p.work_header + 1, 1);
+  if (threadIdx.x == 0) {
+    sh.next_item = atomicAdd(p.work_header + 1, 1);
+    sh.abort = 0;
+  }
   __syncthreads();
   int32_t item = sh.next_item;
-  while (item < total) {
+  while (item < total && !sh.abort) {
     int32_t next = 0;
     if (threadIdx.x == 0) next = atomicAdd(p.work_header + 1, 1);  // in flight during the item
     const int32_t bp = __ldcg(p.work_items + item / p.num_kv_heads);
@@ -569,16 +599,19 @@ inline pa_status encode_pool_map(const void* pool, int32_t num_kv_heads, int32_t
 // of the plan kernel.
 template <bool kMMA, bool kAppend>
 inline pa_status launch_staged_variant(const CUtensorMap& map, const DecodeParams& p, cudaStream_t st) {
-  static int32_t per_sm = -1;
-  if (per_sm < 0) {
+  // once per device: the shared-memory limit and the resident CTAs per SM
+  static PerDevice<int32_t> occupancy;
+  int32_t per_sm = 1;
+  cudaError_t e = occupancy.get(&per_sm, [](int32_t* v) {
     int32_t n = 0;
-    cudaError_t e = cudaFuncSetAttribute(decode_staged_kernel<kMMA, kAppend>,
+    cudaError_t r = cudaFuncSetAttribute(decode_staged_kernel<kMMA, kAppend>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kStagedSmem);
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_staged_kernel<kMMA, kAppend>, 128, kStagedSmem);
-    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode: %s", cudaGetErrorString(e));
-    per_sm = n > 0 ? n : 1;
-  }
+    if (r == cudaSuccess)
+      r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_staged_kernel<kMMA, kAppend>, 128, kStagedSmem);
+    *v = n > 0 ? n : 1;
+    return r;
+  });
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode: %s", cudaGetErrorString(e));
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.blockDim = dim3(128);
@@ -587,18 +620,15 @@ inline pa_status launch_staged_variant(const CUtensorMap& map, const DecodeParam
   if (p.work_items == nullptr) {
     cfg.gridDim = dim3(p.max_partitions, p.num_kv_heads, p.num_seqs);
   } else {
-    int dev = 0, sms = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t most = (int64_t)p.num_seqs * p.max_partitions * p.num_kv_heads;
-    const int64_t resident = (int64_t)per_sm * (sms > 0 ? sms : 148);
+    const int64_t resident = (int64_t)per_sm * device_sm_count();
     cfg.gridDim = dim3((unsigned)(most < resident ? most : resident));
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_staged_kernel<kMMA, kAppend>, map, p);
+  e = cudaLaunchKernelEx(&cfg, decode_staged_kernel<kMMA, kAppend>, map, p);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode: launch failed: %s", cudaGetErrorString(e));
   return PA_OK;
 }

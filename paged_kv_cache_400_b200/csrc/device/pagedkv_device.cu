@@ -2,8 +2,6 @@
 // launches. All kernels live in this one translation unit so they share the
 // per-device error word without relocatable device code.
 #include <cmath>
-#include <cstdlib>
-#include <cstring>
 #include <mutex>
 
 #include "../host/errors.hpp"
@@ -12,14 +10,15 @@
 #include "decode_common.cuh"
 #include "decode_generic.cuh"
 #include "decode_staged.cuh"
-#include "prefill.cuh"
 #include "prefill_tc.cuh"
+#ifdef PA_PREFILL_MMA_SYNC
+#include "prefill.cuh"  // comparison build only: the mma.sync prefill kernel
+#endif
 
 using pagedkv::fail;
 
 namespace {
 
-constexpr int32_t kNumSMs = 148;
 // From this many partitions per sequence the staged decode runs as a
 // persistent grid over a work list (largest partitions first) instead of one
 // CTA per (partition, head, sequence): most grid CTAs of short sequences would
@@ -62,11 +61,42 @@ static_assert(PA_PARTITION_TOKENS % 16 == 0 && PA_PARTITION_TOKENS / 16 <= paged
 int32_t partition_tokens_for(int32_t num_seqs, const pa_pool_desc& pool, int32_t max_seq_len) {
   // PA_PARTITION_TOKENS-token partitions (2048 unless built otherwise: large
   // partitions keep the partial states and their merge small); halve while
-  // the grid would not give every SM a few CTAs, down to 128.
+  // the grid would not give every SM of the current device a few CTAs, down
+  // to 128.
   int32_t S = PA_PARTITION_TOKENS;
   const int64_t pairs = (int64_t)num_seqs * pool.num_kv_heads;
-  while (S > 128 && pairs * ((max_seq_len + S - 1) / S) < 4 * kNumSMs) S /= 2;
+  const int64_t want = 4 * (int64_t)pagedkv::device_sm_count();
+  while (S > 128 && pairs * ((max_seq_len + S - 1) / S) < want) S /= 2;
   return S;
+}
+
+// Host-side checks shared by pa_decode, pa_append_decode and
+// pa_decode_noalloc, in this order: pool, sizes, head group, table width,
+// scale, then (for a non-empty batch) pointers and alignment. The workspace is
+// checked by the caller afterwards.
+pa_status check_decode_args(const char* fn, const void* out, const void* q, const void* kv_pool,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                            int32_t num_seqs, int32_t num_heads, float scale, const pa_pool_desc& pool,
+                            int32_t max_seq_len) {
+  pa_status s = check_pool(pool, fn);
+  if (s != PA_OK) return s;
+  if (num_seqs < 0 || num_heads <= 0 || max_blocks_per_seq <= 0 || max_seq_len < 0)
+    return fail(PA_ERR_INVALID_ARG, "%s: num_seqs %d, num_heads %d, max_blocks %d, max_seq_len %d", fn, num_seqs,
+                num_heads, max_blocks_per_seq, max_seq_len);
+  if (num_heads % pool.num_kv_heads != 0)
+    return fail(PA_ERR_INVALID_ARG, "%s: num_heads %d not a multiple of num_kv_heads %d", fn, num_heads,
+                pool.num_kv_heads);
+  const int32_t G = num_heads / pool.num_kv_heads;
+  if (G > 16) return fail(PA_ERR_UNSUPPORTED, "%s: head group %d > 16", fn, G);
+  if (num_seqs > 65535) return fail(PA_ERR_UNSUPPORTED, "%s: num_seqs %d > 65535", fn, num_seqs);
+  if ((int64_t)max_seq_len > (int64_t)max_blocks_per_seq * PA_BLOCK_SIZE)
+    return fail(PA_ERR_INVALID_ARG, "%s: max_seq_len %d > max_blocks_per_seq * 16", fn, max_seq_len);
+  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "%s: scale is not finite", fn);
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !q || !kv_pool || !block_tables || !seq_lens) return fail(PA_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+  if (!aligned16(out) || !aligned16(q) || !aligned16(kv_pool))
+    return fail(PA_ERR_INVALID_ARG, "%s: out, q and kv_pool must be 16-byte aligned", fn);
+  return PA_OK;
 }
 
 struct WorkspaceLayout {
@@ -170,25 +200,10 @@ pa_status pa_decode(void* out, const void* q, const void* kv_pool, const int32_t
                     int32_t max_blocks_per_seq, const int32_t* seq_lens, int32_t num_seqs,
                     int32_t num_heads, float scale, pa_pool_desc pool, void* workspace,
                     size_t workspace_bytes, int32_t max_seq_len, void* stream) {
-  pa_status s = check_pool(pool, "pa_decode");
-  if (s != PA_OK) return s;
-  if (num_seqs < 0 || num_heads <= 0 || max_blocks_per_seq <= 0 || max_seq_len < 0)
-    return fail(PA_ERR_INVALID_ARG, "pa_decode: num_seqs %d, num_heads %d, max_blocks %d, max_seq_len %d",
-                num_seqs, num_heads, max_blocks_per_seq, max_seq_len);
-  if (num_heads % pool.num_kv_heads != 0)
-    return fail(PA_ERR_INVALID_ARG, "pa_decode: num_heads %d not a multiple of num_kv_heads %d", num_heads,
-                pool.num_kv_heads);
+  pa_status s = check_decode_args("pa_decode", out, q, kv_pool, block_tables, max_blocks_per_seq, seq_lens,
+                                  num_seqs, num_heads, scale, pool, max_seq_len);
+  if (s != PA_OK || num_seqs == 0) return s;
   const int32_t G = num_heads / pool.num_kv_heads;
-  if (G > 16) return fail(PA_ERR_UNSUPPORTED, "pa_decode: head group %d > 16", G);
-  if (num_seqs > 65535) return fail(PA_ERR_UNSUPPORTED, "pa_decode: num_seqs %d > 65535", num_seqs);
-  if ((int64_t)max_seq_len > (int64_t)max_blocks_per_seq * PA_BLOCK_SIZE)
-    return fail(PA_ERR_INVALID_ARG, "pa_decode: max_seq_len %d > max_blocks_per_seq * 16", max_seq_len);
-  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "pa_decode: scale is not finite");
-  if (num_seqs == 0) return PA_OK;
-  if (!out || !q || !kv_pool || !block_tables || !seq_lens)
-    return fail(PA_ERR_INVALID_ARG, "pa_decode: NULL pointer");
-  if (!aligned16(out) || !aligned16(q) || !aligned16(kv_pool))
-    return fail(PA_ERR_INVALID_ARG, "pa_decode: out, q and kv_pool must be 16-byte aligned");
   const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, pool, max_seq_len > 0 ? max_seq_len : 1);
   if (w.total > 0 && (!workspace || workspace_bytes < w.total))
     return fail(PA_ERR_WORKSPACE, "pa_decode: workspace %zu bytes at %p, need %zu", workspace_bytes,
@@ -253,25 +268,10 @@ pa_status pa_append_decode(void* out, const void* q, const void* k_new, const vo
   }
   // Validate exactly as pa_decode does, then launch the decode kernel with the
   // append folded in.
-  pa_status s = check_pool(pool, "pa_append_decode");
-  if (s != PA_OK) return s;
-  if (num_seqs < 0 || num_heads <= 0 || max_blocks_per_seq <= 0 || max_seq_len < 0)
-    return fail(PA_ERR_INVALID_ARG, "pa_append_decode: num_seqs %d, num_heads %d, max_blocks %d, max_seq_len %d",
-                num_seqs, num_heads, max_blocks_per_seq, max_seq_len);
-  if (num_heads % pool.num_kv_heads != 0)
-    return fail(PA_ERR_INVALID_ARG, "pa_append_decode: num_heads %d not a multiple of num_kv_heads %d", num_heads,
-                pool.num_kv_heads);
+  pa_status s = check_decode_args("pa_append_decode", out, q, kv_pool, block_tables, max_blocks_per_seq, seq_lens,
+                                  num_seqs, num_heads, scale, pool, max_seq_len);
+  if (s != PA_OK || num_seqs == 0) return s;
   const int32_t G = num_heads / pool.num_kv_heads;
-  if (G > 16) return fail(PA_ERR_UNSUPPORTED, "pa_append_decode: head group %d > 16", G);
-  if (num_seqs > 65535) return fail(PA_ERR_UNSUPPORTED, "pa_append_decode: num_seqs %d > 65535", num_seqs);
-  if ((int64_t)max_seq_len > (int64_t)max_blocks_per_seq * PA_BLOCK_SIZE)
-    return fail(PA_ERR_INVALID_ARG, "pa_append_decode: max_seq_len %d > max_blocks_per_seq * 16", max_seq_len);
-  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "pa_append_decode: scale is not finite");
-  if (num_seqs == 0) return PA_OK;
-  if (!out || !q || !kv_pool || !block_tables || !seq_lens)
-    return fail(PA_ERR_INVALID_ARG, "pa_append_decode: NULL pointer");
-  if (!aligned16(out) || !aligned16(q) || !aligned16(kv_pool))
-    return fail(PA_ERR_INVALID_ARG, "pa_append_decode: out, q and kv_pool must be 16-byte aligned");
   const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, pool, max_seq_len > 0 ? max_seq_len : 1);
   if (w.total > 0 && (!workspace || workspace_bytes < w.total))
     return fail(PA_ERR_WORKSPACE, "pa_append_decode: workspace %zu bytes at %p, need %zu", workspace_bytes,
@@ -352,15 +352,14 @@ pa_status pa_prefill(void* out, const void* q, const void* kv_pool, const int32_
   p.max_query_len = max_query_len;
   p.num_tokens = num_tokens;
   p.scale_log2 = scale * pagedkv::kLog2e;
-  // tcgen05 kernel; PAGEDKV_PREFILL_KERNEL=mma_sync selects the mma.sync kernel
-  // (same results within rounding; kept for comparison)
-  const char* which = std::getenv("PAGEDKV_PREFILL_KERNEL");
-  if (which && std::strcmp(which, "mma_sync") == 0) {
-    p.tile_tokens = 64 / G;
-    return pagedkv::launch_prefill_bf16_d128(kv_pool, pool.num_blocks, p, num_seqs, (cudaStream_t)stream);
-  }
+#ifdef PA_PREFILL_MMA_SYNC
+  // comparison build: the mma.sync kernel (same results within rounding)
+  p.tile_tokens = 64 / G;
+  return pagedkv::launch_prefill_bf16_d128(kv_pool, pool.num_blocks, p, num_seqs, (cudaStream_t)stream);
+#else
   p.tile_tokens = 128 / G;
   return pagedkv::launch_prefill_tc(kv_pool, pool.num_blocks, p, num_seqs, (cudaStream_t)stream);
+#endif
 }
 
 pa_status pa_copy_blocks(void* kv_pool, const int32_t* src, const int32_t* dst, int32_t n,
@@ -493,6 +492,10 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* kv_
                                        const int32_t* seq_lens, int32_t num_seqs, int32_t num_heads,
                                        float scale, pa_pool_desc pool, int32_t max_seq_len,
                                        void* stream) {
+  // pa_decode's own argument errors come first, then the scratch limit
+  pa_status s = check_decode_args("pa_decode_noalloc", out, q, kv_pool, block_tables, max_blocks_per_seq, seq_lens,
+                                  num_seqs, num_heads, scale, pool, max_seq_len);
+  if (s != PA_OK || num_seqs == 0) return s;
   const size_t need = pa_decode_workspace_size(num_seqs, num_heads, pool, max_seq_len);
   if (need > PA_DECODE_NOALLOC_SCRATCH_BYTES)
     return fail(PA_ERR_WORKSPACE,
@@ -500,7 +503,7 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* kv_
                 "use pa_decode with a workspace",
                 need, (unsigned)PA_DECODE_NOALLOC_SCRATCH_BYTES);
   void* scratch = nullptr;
-  pa_status s = noalloc_scratch(&scratch);
+  s = noalloc_scratch(&scratch);
   if (s != PA_OK) return s;
   return pa_decode(out, q, kv_pool, block_tables, max_blocks_per_seq, seq_lens, num_seqs, num_heads, scale,
                    pool, scratch, PA_DECODE_NOALLOC_SCRATCH_BYTES, max_seq_len, stream);

@@ -19,6 +19,7 @@
 #pragma once
 
 #include "decode_staged.cuh"
+#include "prefill_common.cuh"
 
 namespace pagedkv {
 
@@ -26,23 +27,6 @@ constexpr int kPrefillConsumers = 4;
 constexpr int kPrefillStages = 4;
 constexpr int kPrefillThreads = (kPrefillConsumers + 1) * 32;
 constexpr int kPrefillSmem = kPrefillStages * kStageBytes + 1024;
-
-struct PrefillParams {
-  void* out;                    // [T][H][128] bf16
-  const void* q;                // [T][H][128] bf16
-  const int32_t* block_tables;  // [B][max_blocks]
-  const int32_t* seq_lens;      // [B] KV length, new tokens included
-  const int32_t* query_start;   // [B+1] first q row of each sequence
-  int32_t max_blocks;
-  int32_t num_heads;
-  int32_t num_kv_heads;
-  int32_t group;                // G = H / Hkv, a power of two <= 16
-  int32_t num_blocks;
-  int32_t tile_tokens;          // 64 / G
-  int32_t max_query_len;
-  int32_t num_tokens;           // rows of q / out
-  float scale_log2;
-};
 
 __global__ void __launch_bounds__(kPrefillThreads) prefill_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                   PrefillParams p) {
@@ -262,8 +246,8 @@ inline pa_status launch_prefill_bf16_d128(const void* pool, int32_t num_blocks, 
   CUtensorMap map;
   pa_status s = encode_pool_map(pool, p.num_kv_heads, num_blocks, &map);
   if (s != PA_OK) return s;
-  static cudaError_t attr =
-      cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem);
+  static PerDevice<int32_t> smem_set;
+  cudaError_t attr = set_smem_once(smem_set, prefill_kernel, kPrefillSmem);
   if (attr != cudaSuccess) return fail(PA_ERR_CUDA, "pa_prefill: %s", cudaGetErrorString(attr));
   dim3 grid((p.max_query_len + p.tile_tokens - 1) / p.tile_tokens, p.num_kv_heads, num_seqs);
   prefill_kernel<<<grid, kPrefillThreads, kPrefillSmem, st>>>(map, p);

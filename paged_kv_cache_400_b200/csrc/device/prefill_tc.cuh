@@ -30,7 +30,7 @@
 // Shared memory: Q 2 x 32 KB + 4 x 32 KB KV stages (K and V halves 8 KB each,
 // 128-byte swizzle, the canonical K-major / MN-major UMMA layouts).
 // A one-tile variant (192 threads, 2-stage ring, two CTAs per SM) is kept for
-// comparison (PAGEDKV_PREFILL_QTILES=1).
+// comparison; it is compiled only into a comparison build (PA_PREFILL_QTILES=1).
 // Every wait gives up after 2 s (PA_DEVERR_TIMEOUT); the CTA still frees its
 // tensor memory before it exits. Phase tracking: every mbarrier is waited on at
 // most one completion ahead of the last one its waiter consumed (S and P
@@ -39,9 +39,8 @@
 #pragma once
 
 #include "decode_staged.cuh"
+#include "prefill_common.cuh"
 #include "tcgen05.cuh"
-
-#include <cstdlib>
 
 namespace pagedkv {
 
@@ -55,6 +54,11 @@ constexpr float kTcRescaleLog2 = 8.0f;            // raise the reference max pas
 // kQTiles query tiles of 128 rows share every staged KV tile. Two tiles: one
 // CTA per SM (all 512 tensor-memory columns, 193 KB of shared memory), a
 // 4-deep KV ring; one tile: two CTAs per SM, a 2-deep ring.
+#ifndef PA_PREFILL_QTILES
+#define PA_PREFILL_QTILES 2
+#endif
+static_assert(PA_PREFILL_QTILES == 1 || PA_PREFILL_QTILES == 2, "one or two query tiles per CTA");
+
 template <int kQTiles>
 struct TcConfig {
   static constexpr int kStages = kQTiles == 2 ? 4 : 2;
@@ -461,8 +465,8 @@ inline pa_status launch_prefill_tc_variant(const CUtensorMap& pool_map, const CU
                                            const PrefillParams& p, const uint4* pool, int32_t num_seqs,
                                            cudaStream_t st) {
   using Cfg = TcConfig<kQTiles>;
-  static cudaError_t attr = cudaFuncSetAttribute(prefill_tc_kernel<kQTiles>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+  static PerDevice<int32_t> smem_set;
+  cudaError_t attr = set_smem_once(smem_set, prefill_tc_kernel<kQTiles>, Cfg::kSmem);
   if (attr != cudaSuccess) return fail(PA_ERR_CUDA, "pa_prefill: %s", cudaGetErrorString(attr));
   const int32_t unit_tokens = kQTiles * (128 / p.group);
   dim3 grid((p.max_query_len + unit_tokens - 1) / unit_tokens, p.num_kv_heads, num_seqs);
@@ -480,9 +484,7 @@ inline pa_status launch_prefill_tc(const void* pool, int32_t num_blocks, const P
   s = encode_q_map(p.q, p.num_heads, p.num_tokens, p.group, &q_map);
   if (s != PA_OK) return s;
   const uint4* pool4 = reinterpret_cast<const uint4*>(pool);
-  const char* et = std::getenv("PAGEDKV_PREFILL_QTILES");
-  if (et && std::atoi(et) == 1) return launch_prefill_tc_variant<1>(pool_map, q_map, p, pool4, num_seqs, st);
-  return launch_prefill_tc_variant<2>(pool_map, q_map, p, pool4, num_seqs, st);
+  return launch_prefill_tc_variant<PA_PREFILL_QTILES>(pool_map, q_map, p, pool4, num_seqs, st);
 }
 
 }  // namespace pagedkv

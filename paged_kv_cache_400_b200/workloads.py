@@ -14,6 +14,10 @@ element can be rebuilt on any device from its coordinates alone:
 x_c is an Irwin-Hall(12) variate: mean 0, variance ~1, in [-6, 6), an exact
 multiple of 1/256, so it is the same fp32 number on CPU and GPU and rounds to
 the same bf16 number. It stands in for the N(0, 1) draws the workloads ask for.
+Those values carry at most 11 significant bits, so fp32 products of two of them
+are exact. Cases with full_mantissa=True use y_c = fp32(x_c * 1.05) instead
+(the product formed in fp64, one rounding to fp32: the same number on every
+device), whose fp32 significands are full.
 
 Workloads (sizes follow the decode configurations they are named after):
   tiny      fp32, 4 sequences of length {5, 16, 17, 33} after the append,
@@ -87,26 +91,33 @@ def stream_key(*coords: int) -> int:
     return _s64(k)
 
 
-def values(key, counters: torch.Tensor) -> torch.Tensor:
+FULL_MANTISSA_SCALE = 1.05   # not a dyadic rational: x * 1.05 fills the fp32 significand
+
+
+def values(key, counters: torch.Tensor, full_mantissa: bool = False) -> torch.Tensor:
     """Irwin-Hall(12) values (fp32) at the given int64 counters of stream `key`
-    (an int, or an int64 tensor of keys broadcast against the counters)."""
+    (an int, or an int64 tensor of keys broadcast against the counters);
+    with full_mantissa, each value times 1.05 rounded once to fp32."""
     n = counters.to(torch.int64) * 2
     h1 = _mix(n * _GAMMA + key)
     h2 = _mix((n + 1) * _GAMMA + key)
-    s = torch.zeros_like(h1)
-    for i in range(8):
-        s += _shr(h1, 8 * i) & 0xFF
-    for i in range(4):
-        s += _shr(h2, 8 * i) & 0xFF
-    return (s.to(torch.float32) + 6.0) / 256.0 - 6.0
+    shape = h1.shape
+    # the 8 bytes of h1 and the low 4 bytes of h2 (little-endian byte views)
+    b1 = h1.reshape(-1).contiguous().view(torch.uint8).view(-1, 8)
+    b2 = h2.reshape(-1).contiguous().view(torch.uint8).view(-1, 8)[:, :4]
+    s = (b1.sum(dim=1, dtype=torch.int32) + b2.sum(dim=1, dtype=torch.int32)).reshape(shape)
+    x = (s.to(torch.float32) + 6.0) / 256.0 - 6.0
+    if full_mantissa:
+        x = (x.to(torch.float64) * FULL_MANTISSA_SCALE).to(torch.float32)
+    return x
 
 
 def value_block(key: int, shape, offset: int = 0, device="cpu",
-                dtype=torch.float32) -> torch.Tensor:
+                dtype=torch.float32, full_mantissa: bool = False) -> torch.Tensor:
     """Values at counters offset .. offset+prod(shape)-1, row-major in `shape`."""
     n = int(np.prod(shape))
     c = torch.arange(offset, offset + n, dtype=torch.int64, device=device)
-    return values(key, c).to(dtype).reshape(shape)
+    return values(key, c, full_mantissa).to(dtype).reshape(shape)
 
 
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
@@ -144,6 +155,7 @@ class DecodeCase:
     table_width: int
     max_seq_len: int
     info: dict = field(default_factory=dict)
+    full_mantissa: bool = False   # values x * 1.05 (full fp32 significands)
 
     @property
     def pool_shape(self):
@@ -158,7 +170,7 @@ class DecodeCase:
             b1 = min(b0 + chunk_blocks, self.num_blocks)
             pool[b0:b1] = value_block(key, (b1 - b0,) + self.pool_shape[1:],
                                       offset=b0 * per_block, device=device,
-                                      dtype=pool.dtype)
+                                      dtype=pool.dtype, full_mantissa=self.full_mantissa)
         return pool
 
     def pool_blocks(self, block_ids, device="cpu") -> torch.Tensor:
@@ -167,20 +179,21 @@ class DecodeCase:
         key = stream_key(self.seed, TAG_POOL)
         ids = torch.as_tensor(np.asarray(block_ids, dtype=np.int64), device=device)
         c = ids[:, None] * per_block + torch.arange(per_block, device=device)[None, :]
-        return values(key, c).to(TORCH_DTYPE[self.dtype]).reshape(
+        return values(key, c, self.full_mantissa).to(TORCH_DTYPE[self.dtype]).reshape(
             (len(block_ids),) + self.pool_shape[1:])
 
     def make_q(self, device="cpu") -> torch.Tensor:
         return value_block(stream_key(self.seed, TAG_Q),
                            (len(self.batch), self.num_heads, self.head_dim),
-                           device=device, dtype=TORCH_DTYPE[self.dtype])
+                           device=device, dtype=TORCH_DTYPE[self.dtype],
+                           full_mantissa=self.full_mantissa)
 
     def make_kv_new(self, device="cpu"):
         shape = (len(self.batch), self.num_kv_heads, self.head_dim)
         k = value_block(stream_key(self.seed, TAG_K), shape, device=device,
-                        dtype=TORCH_DTYPE[self.dtype])
+                        dtype=TORCH_DTYPE[self.dtype], full_mantissa=self.full_mantissa)
         v = value_block(stream_key(self.seed, TAG_V), shape, device=device,
-                        dtype=TORCH_DTYPE[self.dtype])
+                        dtype=TORCH_DTYPE[self.dtype], full_mantissa=self.full_mantissa)
         return k, v
 
 
@@ -197,10 +210,12 @@ def _decode_case_from_lens(name, seed, lens_after, num_blocks, num_heads, num_kv
                       info={"seq_lens_after_append": [int(x) for x in lens_after]})
 
 
-def tiny_case(seed: int = 0) -> DecodeCase:
+def tiny_case(seed: int = 0, full_mantissa: bool = False) -> DecodeCase:
     rng = np.random.default_rng(seed)
-    return _decode_case_from_lens("tiny_fp32", seed, [5, 16, 17, 33], 64, 2, 2, 64,
-                                  "f32", 1.0 / 8.0, 4, 64, rng)
+    case = _decode_case_from_lens("tiny_fp32_full" if full_mantissa else "tiny_fp32", seed,
+                                  [5, 16, 17, 33], 64, 2, 2, 64, "f32", 1.0 / 8.0, 4, 64, rng)
+    case.full_mantissa = full_mantissa
+    return case
 
 
 def mha_case(seed: int = 0, batch: int = 64) -> DecodeCase:
@@ -223,14 +238,16 @@ def gqa_case(seed: int = 0, batch: int = 256) -> DecodeCase:
 
 
 def custom_case(name, seed, lens_after, num_blocks, num_heads, num_kv_heads, head_dim,
-                dtype, table_width, max_seq_len, scale=None) -> DecodeCase:
+                dtype, table_width, max_seq_len, scale=None, full_mantissa=False) -> DecodeCase:
     """A decode step with caller-chosen lengths (edge cases, small variants)."""
     rng = np.random.default_rng(seed + 303)
     if scale is None:
         scale = head_dim ** -0.5
-    return _decode_case_from_lens(name, seed, list(lens_after), num_blocks, num_heads,
+    case = _decode_case_from_lens(name, seed, list(lens_after), num_blocks, num_heads,
                                   num_kv_heads, head_dim, dtype, scale, table_width,
                                   max_seq_len, rng)
+    case.full_mantissa = full_mantissa
+    return case
 
 
 def prefix_case(seed: int = 0) -> DecodeCase:
@@ -296,6 +313,7 @@ class PrefillCase:
     query_lens: list
     table_width: int
     info: dict = field(default_factory=dict)
+    full_mantissa: bool = False   # prefill inputs are bf16: the short values round the same
 
     pool_shape = DecodeCase.pool_shape
     make_pool = DecodeCase.make_pool

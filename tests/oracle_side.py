@@ -98,9 +98,13 @@ def oracle_compute(x):
     return oa.paged_decode(x["q"], x["pool"], x["tables"], x["lens"], x["scale"], x["dtype"])
 
 
-def oracle_outputs(case, ost: OracleStep, sample):
-    """fp64 oracle output for batch rows `sample` ([len(sample)][H][D])."""
-    return oracle_compute(oracle_inputs(case, ost, sample))
+def oracle_outputs(case, ost: OracleStep, sample, chunk: int = 16):
+    """fp64 oracle output for batch rows `sample` ([len(sample)][H][D]), built
+    `chunk` rows at a time (each chunk's pool holds only its blocks)."""
+    sample = list(sample)
+    parts = [oracle_compute(oracle_inputs(case, ost, sample[i:i + chunk]))
+             for i in range(0, len(sample), chunk)]
+    return np.concatenate(parts) if parts else np.zeros((0, case.num_heads, case.head_dim))
 
 
 def tolerance_ok(case, out_gpu: np.ndarray, ref: np.ndarray):

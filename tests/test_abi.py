@@ -68,6 +68,26 @@ def test_decode_rejects_bad_arguments_on_host():
     assert L.pa_decode(None, None, None, None, 4, None, 0, 2, 0.1, p, None, 0, 16, None) == 0
 
 
+def test_noalloc_reports_argument_errors_before_its_size_limit():
+    """pa_decode_noalloc returns pa_decode's own argument errors even for a
+    shape beyond its fixed array; only valid arguments reach the size check."""
+    L = bd.lib()
+    vp = C.c_void_p(16)  # never dereferenced: rejected before use
+    big = pool(num_blocks=1 << 20, heads=8)
+    B, width, max_len = 1024, 2048, 32768   # partials far beyond the fixed array
+    assert L.pa_decode_workspace_size(B, 32, big, max_len) > (32 << 20)
+    call = lambda H, desc=big, mb=width, ml=max_len, scale=0.1: L.pa_decode_noalloc(
+        vp, vp, vp, vp, mb, vp, B, H, scale, desc, ml, None)
+    assert call(36) == 1                          # num_heads not a multiple of num_kv_heads
+    assert call(8 * 32) == 2                      # head group 32
+    assert call(32, mb=1024) == 1                 # max_seq_len beyond max_blocks * 16
+    assert call(32, scale=float("nan")) == 1
+    assert call(32, desc=pool(num_blocks=1 << 20, heads=8, dim=96)) == 2
+    assert call(32) == 9                          # valid arguments: the size limit
+    assert b"fixed array" in L.pa_last_error()
+    assert L.pa_decode_noalloc(None, None, None, None, 4, None, 0, 2, 0.1, pool(), 16, None) == 0
+
+
 def test_prefill_rejects_bad_arguments_on_host():
     L = bd.lib()
     vp = C.c_void_p(16)  # never dereferenced: rejected before use

@@ -68,23 +68,66 @@ def test_tiny_fp32_full():
     assert np.array_equal(storage_bits(pool).view(np.uint32), ref_pool.view(np.uint32))
 
 
-def test_mha_sampled():
-    case = wl.mha_case(0)
-    lens = case.info["seq_lens_after_append"]
-    sample = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 0, 1, 17, 63})
-    check_case(case, sample)
+def test_tiny_fp32_full_mantissa():
+    """The tiny fp32 config with inputs whose fp32 significands are full (x *
+    1.05 rounded once), so products in q.k and p.v round: held to the same
+    2e-5 relative bar, and the appended pool bit-exact."""
+    case = wl.tiny_case(0, full_mantissa=True)
+    prep, pool, out, err = check_case(case)
+    from oracle import attention as oa
+    ref_pool = storage_bits(case.make_pool("cpu")).copy()
+    k, v = case.make_kv_new("cpu")
+    oa.reshape_and_cache(ref_pool, storage_bits(k), storage_bits(v), prep.slot_mapping)
+    assert np.array_equal(storage_bits(pool).view(np.uint32), ref_pool.view(np.uint32))
 
 
-def test_gqa_sampled():
+@pytest.mark.parametrize("dim,heads,kv", [(64, 2, 2), (128, 8, 2), (64, 6, 1), (128, 32, 8)])
+def test_fp32_full_mantissa_shapes(dim, heads, kv):
+    """fp32 with full-significand inputs across tiles, ragged tails and several
+    partitions (lengths 1 to 4096 on a 4096 bound), against the 2e-5 bar."""
+    lens = [1, 15, 16, 17, 33, 129, 511, 513, 1025, 2048, 3001, 4096]
+    case = wl.custom_case(f"f32full_{dim}_{heads}_{kv}", 8, lens, 1024, heads, kv, dim, "f32", 256, 4096,
+                          full_mantissa=True)
+    check_case(case)
+
+
+def test_mha_every_sequence():
+    """The Llama-2-7B-shaped MHA config at its stated size, all 64 sequences
+    compared element by element with the fp64 oracle."""
+    check_case(wl.mha_case(0))
+
+
+def test_gqa_every_sequence():
+    """The Llama-3-8B-shaped GQA batch of 256 at its stated size, every
+    sequence compared element by element with the fp64 oracle."""
+    check_case(wl.gqa_case(0))
+
+
+def test_gqa_fused_step_every_sequence():
+    """The same batch through pa_append_decode (the benchmarked step): every
+    sequence against the oracle, and the appended pool rows bit-exact."""
     case = wl.gqa_case(0)
-    lens = case.info["seq_lens_after_append"]
-    sample = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 0, 5, 100, 255})
-    check_case(case, sample)
+    prep = prepare_decode_step(case)
+    ost = oracle_indices(case)
+    pool = case.make_pool(DEV)
+    q = case.make_q(DEV)
+    k, v = case.make_kv_new(DEV)
+    out = torch.empty_like(q)
+    slots = torch.from_numpy(prep.slot_mapping).to(DEV)
+    ws = pk.alloc_workspace(len(case.batch), case.num_heads, pool, case.max_seq_len)
+    pk.pa_append_decode(out, q, k, v, pool, slots, torch.from_numpy(prep.block_tables).to(DEV),
+                        torch.from_numpy(prep.seq_lens).to(DEV), case.scale, case.max_seq_len, ws)
+    assert pk.pa_get_device_error() == 0
+    blk, row = slots // 16, slots % 16
+    assert torch.equal(pool[blk, 0, :, row, :], k) and torch.equal(pool[blk, 1, :, row, :], v)
+    ref = oracle_outputs(case, ost, range(len(case.batch)))
+    ok, err = tolerance_ok(case, out.float().cpu().numpy().astype(np.float64), ref)
+    assert ok, err
 
 
 def test_shared_prefix_with_copy_on_write():
     case = wl.prefix_case(0)
-    sample = [0, 7, 31, 32, 33, 34, 35, 63]  # prefix sharers and one sampled prompt
+    sample = None  # every sequence: the 32 prefix sharers and the 8 x 4 samples
     prep, pool, out, err = check_case(case, sample)
     assert len(prep.cow_src) == 24
     # copied blocks are bit-identical to their sources except the appended row

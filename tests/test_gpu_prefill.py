@@ -10,6 +10,7 @@ import pytest
 import torch
 
 import paged_kv_cache_400_b200 as pk
+from paged_kv_cache_400_b200 import binding as bd
 from paged_kv_cache_400_b200 import workloads as wl
 from paged_kv_cache_400_b200.scenario import prepare_prefill_step
 
@@ -21,17 +22,13 @@ DEV = "cuda"
 
 
 @pytest.fixture(autouse=True, params=["tcgen05", "tcgen05_1tile", "mma_sync"])
-def prefill_kernel(request, monkeypatch):
-    """Every test runs on each prefill kernel: tcgen05 with two query tiles per
-    CTA (the default), tcgen05 with one (PAGEDKV_PREFILL_QTILES=1), and the
-    mma.sync kernel (PAGEDKV_PREFILL_KERNEL=mma_sync)."""
-    monkeypatch.delenv("PAGEDKV_PREFILL_KERNEL", raising=False)
-    monkeypatch.delenv("PAGEDKV_PREFILL_QTILES", raising=False)
-    if request.param == "mma_sync":
-        monkeypatch.setenv("PAGEDKV_PREFILL_KERNEL", "mma_sync")
-    elif request.param == "tcgen05_1tile":
-        monkeypatch.setenv("PAGEDKV_PREFILL_QTILES", "1")
-    return request.param
+def prefill_kernel(request):
+    """Every test runs on each prefill kernel: the product library's tcgen05
+    kernel, and the two comparison builds (tcgen05 with one query tile per
+    CTA, and the mma.sync kernel), each a library of its own."""
+    variant = {"tcgen05": None, "tcgen05_1tile": "prefill_1tile", "mma_sync": "prefill_mma_sync"}[request.param]
+    with bd.use_variant(variant):
+        yield request.param
 
 
 def device_prefill(case, prep, pool=None):

@@ -92,6 +92,73 @@ def test_trace_with_preemption_matches_oracle():
     eng.close()
 
 
+def test_full_size_trace_matches_oracle():
+    """The continuous-batching config at its stated size: 2000 requests,
+    Poisson(50) arrivals per step, prompts U[16, 1024], outputs geometric (mean
+    200, cap 2048), one 40 000-block pool (one layer: every layer runs the same
+    calls on a pool of its own). Every step's running set, lengths, block
+    tables, decode slots and prompt slots equal the oracle scheduler's; at least
+    40 (step, request) attention rows are compared with the fp64 oracle, among
+    them requests right after a preemption and re-admission (their prompt and
+    generated tokens' K/V rewritten by recompute) and again a few steps later."""
+    trace = wl.trace_case(seed=0, num_layers=1)
+    eng = DecodeEngine(trace.num_blocks, trace.num_layers, trace.num_heads, trace.num_kv_heads,
+                       trace.head_dim, trace.arrival_step, trace.prompt_len, trace.output_len,
+                       trace.table_width, trace.scale, DEV)
+    obm = OracleBlockManager(trace.num_blocks)
+    osch = OracleScheduler(obm, trace.arrival_step, trace.prompt_len, trace.output_len, trace.table_width)
+    rng = np.random.default_rng(3)
+    preempted_ever, follow = set(), {}
+    checked = readmit_checked = later_checked = steps = 0
+    while True:
+        idx = eng.schedule()
+        o = osch.step()
+        steps += 1
+        assert idx.running.tolist() == o["running"]
+        assert idx.seq_lens.tolist() == o["seq_lens"]
+        assert idx.decode_slots.tolist() == o["decode_slots"]
+        assert idx.prompt_slots.tolist() == o["prompt_slots"]
+        assert idx.prompt_seqs.tolist() == o["prompt_seqs"]
+        if len(idx.running):
+            assert np.array_equal(idx.block_tables, np.asarray(o["block_tables"], np.int32))
+        readmitted = [r for r in o["prompt_seqs"] if r in preempted_ever]
+        preempted_ever.update(o["preempted"])
+        if len(idx.running):
+            inputs = [layer_inputs(trace, eng, idx, 0, DEV)]
+            outs = eng.run_layers(idx, inputs)
+            row_of = {int(r): i for i, r in enumerate(idx.running)}
+            picks = []
+            if readmit_checked < 16:
+                for r in readmitted[:2]:
+                    picks.append((r, "readmit"))
+                    follow.setdefault(r, idx.step + 5)
+            for r, at in list(follow.items()):
+                if at == idx.step and r in row_of:
+                    picks.append((r, "later"))
+                    del follow[r]
+            if idx.step % 50 == 0:
+                picks.append((int(idx.running[int(rng.integers(len(idx.running)))]), "random"))
+            if picks:
+                got = outs[0].float().cpu().numpy()
+                for r, why in picks:
+                    i = row_of[r]
+                    L = o["seq_lens"][i]
+                    ref = oracle_attention(trace, 0, idx.step, r, o["block_tables"][i][:(L + 15) // 16], L)
+                    err = float(np.abs(got[i] - ref).max())
+                    assert err <= 1e-2, (idx.step, r, why, err)
+                    checked += 1
+                    readmit_checked += why == "readmit"
+                    later_checked += why == "later"
+        if idx.done:
+            break
+    import paged_kv_cache_400_b200 as pk
+    assert pk.pa_get_device_error() == 0
+    eng.close()
+    assert steps > 1000 and len(preempted_ever) > 0
+    assert checked >= 40 and readmit_checked >= 10 and later_checked >= 5, \
+        (checked, readmit_checked, later_checked)
+
+
 def test_graphed_layer_loop_matches_oracle():
     """The same trace with each step's decode over all layers replayed as a CUDA
     graph per batch bucket (padded rows inert)."""
