@@ -23,7 +23,6 @@ import argparse
 import hashlib
 import json
 import os
-import re
 import statistics
 import sys
 import threading
@@ -37,7 +36,7 @@ sys.path.insert(0, ROOT)
 METRIC = "paged decode-attn tokens/s; KV-read HBM GB/s as fraction of ~8 TB/s peak"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "pa_decode_gqa_b256.md")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "pa_decode_gqa_b256.json")
 
 
 def parse_args():
@@ -70,6 +69,12 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="bounded oracle sample for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-cpu-seconds", type=float, default=4.0,
+                    help="bounded oracle sample of the chunked-prefill leg")
+    ap.add_argument("--no-prefill-leg", action="store_true",
+                    help="gqa: skip the chunked-prefill measurement added to the line")
+    ap.add_argument("--kv-util-jsonl", default=None,
+                    help="trace: write each step's KV-cache utilisation record to this file")
     return ap.parse_args()
 
 
@@ -178,22 +183,32 @@ class ClockSampler:
             self._stop.set()
             self._t.join()
 
-    def summary(self, t0, t1):
+    def summary(self, t0, t1, timed=None):
+        """Clocks over the window [t0, t1] (the timed region plus the loops
+        measured right after it on the same data); `timed` = (start, end) of
+        the timed region itself, whose own sample count is reported too."""
         if not self.ok:
             return {"error": getattr(self, "err", "nvml unavailable")}
         inside = [s for s in self.samples if t0 <= s[0] <= t1]
-        note = "sampled during the timed region"
+        note = ("sampled every 10 ms from the start of the timed region to the end of the "
+                "comparison and end-to-end loops that follow it")
         if not inside:
             inside = self.samples[-5:]
-            note = "timed region shorter than the sampling period: last samples before its end"
+            note = "window shorter than the sampling period: last samples before its end"
         reasons = set()
         for _, _, rs in inside:
             for bit, name in self.REASONS.items():
                 if rs & bit:
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(m for _, m, _ in inside) if inside else None,
-                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
-                "samples": len(inside), "note": note}
+        out = {"sm_mhz": statistics.median(m for _, m, _ in inside) if inside else None,
+               "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+               "samples": len(inside), "window_s": t1 - t0, "note": note}
+        if timed is not None:
+            tin = [s for s in self.samples if timed[0] <= s[0] <= timed[1]]
+            out["timed_region_samples"] = len(tin)
+            if tin:
+                out["timed_region_sm_mhz"] = statistics.median(m for _, m, _ in tin)
+        return out
 
 
 DECODE_KERNEL_SOURCES = ("common.cuh", "decode_common.cuh", "decode_staged.cuh", "ptx.cuh")
@@ -215,18 +230,18 @@ def kernel_source_digest(sources=None):
 
 
 def recorded_traffic(path=None, sources=None):
-    """ncu DRAM bytes per launch recorded in profiles/, if taken on this source."""
+    """ncu DRAM bytes per launch recorded in profiles/<kernel>_<workload>.json
+    (beside the summary of the same capture), if taken on this source."""
     try:
-        text = open(path or TRAFFIC_FILE).read()
-    except OSError:
-        return None, "no ncu summary"
-    m = re.search(r"kernel_source_digest:\s*([0-9a-f]+)", text)
-    t = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-    if not (m and t):
-        return None, "summary lacks digest or traffic"
-    if m.group(1) != kernel_source_digest(sources):
+        with open(path or TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None, "no ncu record"
+    if "kernel_source_digest" not in rec or "dram_bytes_per_launch" not in rec:
+        return None, "record lacks digest or traffic"
+    if rec["kernel_source_digest"] != kernel_source_digest(sources):
         return None, "kernel changed since the ncu capture"
-    return int(t.group(1)), "ncu capture"
+    return int(rec["dram_bytes_per_launch"]), "ncu capture (%s)" % rec.get("captured", "?")
 
 
 def measured_peak():
@@ -342,6 +357,7 @@ def run_ours(args, rank, world, dist):
     ws = pk.alloc_workspace(B, H, pool, case.max_seq_len)
     S = pk.pa_decode_partition_tokens(B, H, pool, case.max_seq_len)
     parts = [(int(n) + S - 1) // S for n in prep.seq_lens]
+    max_parts = (case.max_seq_len + S - 1) // S   # partitions the launch is sized for
     nbytes = algorithmic_bytes(case, prep, parts, max(parts))
     stream = torch.cuda.current_stream()
     cow_src = torch.from_numpy(prep.cow_src).to(dev) if len(prep.cow_src) else None
@@ -380,7 +396,6 @@ def run_ours(args, rank, world, dist):
     wall1 = time.perf_counter()
     if dist is not None:
         dist.barrier()
-    sampler.stop()
     # the same step as separate calls, for comparison
     total_sep, (_, app_ms, dec_ms) = timed_loop(K, stream, [cow, append, decode])
     assert pk.pa_get_device_error() == 0
@@ -470,8 +485,15 @@ def run_ours(args, rank, world, dist):
             out_done[b].record(s_out)
     torch.cuda.synchronize()
     p1 = time.perf_counter()
+    sampler.stop()
     e2e_s = max_over_ranks((p1 - p0) / E, dist, dev)
     assert pk.pa_get_device_error() == 0
+
+    # the chunked-prefill leg (the step on the other side of decode), every rank
+    prefill_line = None
+    if args.workload == "gqa" and not args.no_prefill_leg:
+        prefill_line = measure_prefill(args, rank, world, dist, True, max(K, 10), args.warmup,
+                                       None if args.no_cpu_baseline else args.prefill_cpu_seconds)
 
     if rank != 0:
         return
@@ -506,8 +528,12 @@ def run_ours(args, rank, world, dist):
                            "decode_avg_ms": dec_avg,
                            "decode_frac_of_measured": nbytes["decode"] / (dec_avg / 1e3) / 1e9 / peak,
                            "value": world * B / (total_sep / K / 1e3)},
-        "gpu_launches": K * (1 + (1 if max(parts) > 1 else 0) + (1 if cow_src is not None else 0)),
-        "clocks": sampler.summary(wall0, wall1),
+        # per step: the decode kernel, the partition merge when the bound
+        # allows several partitions, the plan kernel from 4 partitions on (the
+        # work-list path), and the copy-on-write copy when there are pairs
+        "gpu_launches": K * (1 + (1 if max_parts > 1 else 0) + (1 if max_parts >= 4 else 0)
+                             + (1 if cow_src is not None else 0)),
+        "clocks": sampler.summary(wall0, p1, timed=(wall0, wall1)),
         "e2e": {"value": world * B / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "note": "per step: host table packing (pa_bm_pack), H2D of q/k/v/slots/tables/lens "
@@ -523,6 +549,8 @@ def run_ours(args, rank, world, dist):
         ub = uniq * 2 * case.num_kv_heads * 16 * D * 2
         line["unique_kv_bytes"] = ub
         line["unique_kv_gbs"] = ub / (ms_per_step / 1e3) / 1e9
+    if prefill_line is not None:
+        line["chunked_prefill"] = prefill_line
     if not args.no_cpu_baseline and world == 1:
         done, el = oracle_sample(case, args.cpu_seconds)
         line["cpu_baseline"] = {
@@ -539,6 +567,57 @@ def run_ours(args, rank, world, dist):
             line["cpu_baseline"]["one_core_value"] = None
             line["cpu_baseline"]["one_core_error"] = repr(e)
     print(json.dumps(line), flush=True)
+
+
+def trace_oracle_scheduler(tr, caching, swap_host_blocks):
+    """The oracle scheduler over the trace's requests, configured as the run."""
+    sys.path.insert(0, ROOT)
+    from oracle.block_manager import OracleBlockManager
+    from oracle.scheduler import OracleScheduler
+    bm = OracleBlockManager(tr.num_blocks)
+    if caching:
+        bm.set_prefix_caching(True)
+    sch = OracleScheduler(bm, tr.arrival_step, tr.prompt_len, tr.output_len, tr.table_width)
+    if caching:
+        sch.set_prompt_tokens(tr.prompt_tokens)
+    if swap_host_blocks:
+        sch.set_swap(swap_host_blocks)
+    return sch
+
+
+def trace_oracle_plan(tr, caching, swap_host_blocks, n_samples, rows_per_sample, seed):
+    """The oracle's side of the trace measurement. Replays the whole trace on
+    the oracle scheduler (timed: the integer half of the oracle, in full), then
+    picks `n_samples` seeded (step, layer) samples and, per sample, up to
+    `rows_per_sample` running requests, and replays once more (untimed) to keep
+    those steps' requests, lengths and block tables. Returns (replay seconds,
+    steps, {step: (layer, [(row, request, length, table)])})."""
+    t0 = time.perf_counter()
+    sch = trace_oracle_scheduler(tr, caching, swap_host_blocks)
+    running = []
+    while True:
+        o = sch.step()
+        running.append(len(o["running"]))
+        if o["done"]:
+            break
+    replay_s = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    busy = [i for i, n in enumerate(running) if n > 0]
+    steps = sorted(int(x) for x in rng.choice(busy, size=min(n_samples, len(busy)), replace=False))
+    plan = {st: int(rng.integers(tr.num_layers)) for st in steps}
+    picks = {}
+    sch = trace_oracle_scheduler(tr, caching, swap_host_blocks)
+    while True:
+        o = sch.step()
+        st = o["step"]
+        if st in plan:
+            n = len(o["running"])
+            rows = sorted(int(x) for x in rng.choice(n, size=min(rows_per_sample, n), replace=False))
+            picks[st] = (plan[st], [(i, o["running"][i], o["seq_lens"][i],
+                                     o["block_tables"][i][:(o["seq_lens"][i] + 15) // 16]) for i in rows])
+        if o["done"]:
+            break
+    return replay_s, len(running), picks
 
 
 def run_trace(args, rank, world):
@@ -574,6 +653,17 @@ def run_trace(args, rank, world):
         from paged_kv_cache_400_b200.engine import GraphedLayers
         graphed = GraphedLayers(eng, max_batch=1280)
     stream = torch.cuda.current_stream()
+    # the oracle's half: full scheduler replay (timed) and the sampled steps
+    oracle_on = not args.no_cpu_baseline and world == 1
+    if oracle_on:
+        replay_s, oracle_steps, picks = trace_oracle_plan(tr, caching, args.swap_host_blocks, 20, 2,
+                                                          args.seed + 17)
+    else:
+        picks = {}
+    got_rows = {}
+    util_log = open(args.kv_util_jsonl, "w") if args.kv_util_jsonl else None
+    utils, occupancy = [], []
+    slots_held = 0
     events = []
     tokens = kv_tokens = prompt_tokens = steps = preempted = cached_tokens = peak_batch = 0
     swap_blocks = 0
@@ -598,16 +688,32 @@ def run_trace(args, rank, world):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             if graphed is not None:
-                graphed.run(idx, inputs, stacked)
+                outs = graphed.run(idx, inputs, stacked)
             else:
-                eng.run_layers(idx, inputs)
+                outs = eng.run_layers(idx, inputs)
             e1.record(stream)
             torch.cuda.synchronize()
             e2e_s += (t1 - t0) + (time.perf_counter() - t2)
             events.append((e0, e1))
+            if idx.step in picks:
+                layer, rows = picks[idx.step]
+                got_rows[idx.step] = outs[layer][[r for r, _, _, _ in rows]].float().cpu().numpy()
             tokens += n
-            kv_tokens += int(idx.seq_lens.astype(np.int64).sum())
+            lens_sum = int(idx.seq_lens.astype(np.int64).sum())
+            kv_tokens += lens_sum
             prompt_tokens += len(idx.prompt_slots)
+            # KV-cache utilisation: token slots holding a running request's KV
+            # over the slots of the distinct blocks those requests hold
+            held = np.unique(idx.block_tables[idx.block_tables >= 0])
+            util = lens_sum / (16.0 * len(held))
+            occ = (tr.num_blocks - idx.record.num_free_blocks) / tr.num_blocks
+            utils.append(util)
+            occupancy.append(occ)
+            slots_held += 16 * len(held)
+            if util_log is not None:
+                util_log.write(json.dumps({"step": int(idx.step), "running": n, "kv_tokens": lens_sum,
+                                           "blocks_held": int(len(held)), "kv_util": util,
+                                           "pool_occupancy": occ}) + "\n")
         steps += 1
         preempted += idx.record.preempted
         cached_tokens += int(idx.prompt_starts.sum())
@@ -617,6 +723,8 @@ def run_trace(args, rank, world):
             break
     wall1 = time.perf_counter()
     sampler.stop()
+    if util_log is not None:
+        util_log.close()
     assert pk.pa_get_device_error() == 0
     gpu_s = sum(a.elapsed_time(b) for a, b in events) / 1e3
     eng.close()
@@ -645,7 +753,40 @@ def run_trace(args, rank, world):
         "e2e": {"value": tokens / e2e_s, "unit": "tokens/s",
                 "note": "pa_sched_step + index H2D + layer loops, wall clock; input generation excluded"},
         "wall_s": wall1 - wall0, "clocks": sampler.summary(wall0, wall1),
+        "kv_util": {"mean": float(np.mean(utils)), "min": float(np.min(utils)),
+                    "over_all_steps": kv_tokens / max(1, slots_held),
+                    "pool_occupancy_mean": float(np.mean(occupancy)),
+                    "definition": "per step: KV tokens of the running requests / (16 x distinct blocks "
+                                  "they hold); pool_occupancy = blocks held / pool blocks",
+                    "per_step_jsonl": args.kv_util_jsonl},
     }
+    if oracle_on:
+        # parity and timing of the oracle's attention on the sampled rows
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        from oracle_side import oracle_trace_row
+        att_s, att_tokens, max_err, n_rows = 0.0, 0, 0.0, 0
+        for st, (layer, rows) in picks.items():
+            for j, (_, req, length, table) in enumerate(rows):
+                ref, dt = oracle_trace_row(tr, layer, st, req, table, length)
+                max_err = max(max_err, float(np.abs(got_rows[st][j] - ref).max()))
+                att_s += dt
+                att_tokens += length
+                n_rows += 1
+        assert max_err <= 1e-2, f"trace: sampled decode rows differ from the oracle by {max_err}"
+        # oracle time of the whole run: the replay (measured in full) plus the
+        # attention of every (step, layer, request), extrapolated from the
+        # sampled rows by their KV tokens
+        att_total = att_s / att_tokens * (kv_tokens * tr.num_layers)
+        line["parity"] = {"sampled_steps": len(picks), "rows": n_rows, "max_abs_err": max_err, "bar": 1e-2,
+                          "oracle": "fp64 append + gather through the oracle scheduler's own tables"}
+        line["cpu_baseline"] = {
+            "value": tokens / (replay_s + att_total), "unit": "tokens/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"oracle scheduler replay of the whole trace timed in full ({replay_s:.2f} s, "
+                      f"{oracle_steps} steps); fp64 attention timed on {n_rows} rows of {len(picks)} seeded "
+                      f"(step, layer) samples ({att_s:.2f} s for {att_tokens} KV tokens) and extrapolated "
+                      f"by KV tokens to every request of every step and layer ({att_total:.0f} s)",
+            "replay_s": replay_s, "attention_s_extrapolated": att_total}
     print(json.dumps(line), flush=True)
 
 
@@ -690,10 +831,20 @@ def oracle_prefill_sample(case, seconds, rng_seed=0):
 
 
 def run_prefill(args, rank, world, dist):
+    """The prefill workloads as the benchmark line (see measure_prefill)."""
+    line = measure_prefill(args, rank, world, dist, args.workload == "chunked_prefill", args.steps,
+                           args.warmup, None if args.no_cpu_baseline else args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def measure_prefill(args, rank, world, dist, chunked, K, warmup, cpu_seconds):
     """One prefill step per iteration: append every new token's K/V into its
     slot (pa_reshape_and_cache), then causal paged attention of the new tokens
-    (pa_prefill). Reports new tokens per second and the attention kernel's
-    TFLOP/s against the measured bf16 tensor peak."""
+    (pa_prefill). Returns (on rank 0; None elsewhere) the line: new tokens per
+    second, the attention kernel's TFLOP/s against the measured bf16 tensor
+    peak, the end-to-end rate from host buffers and, with cpu_seconds, the
+    oracle on a bounded sample."""
     import torch
 
     import paged_kv_cache_400_b200 as pk
@@ -703,7 +854,6 @@ def run_prefill(args, rank, world, dist):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    chunked = args.workload == "chunked_prefill"
     pb = args.prefill_batch
     case = (wl.chunked_prefill_case(args.seed + rank, batch=pb) if chunked
             else wl.prefill_case(args.seed + rank, batch=pb))
@@ -726,11 +876,10 @@ def run_prefill(args, rank, world, dist):
     def attend():
         pk.pa_prefill(out, q, pool, bt, sl, qs, case.scale, mq)
 
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         append()
         attend()
     assert pk.pa_get_device_error() == 0
-    K = args.steps
     sampler = ClockSampler(local)
     sampler.start()
     if dist is not None:
@@ -741,7 +890,6 @@ def run_prefill(args, rank, world, dist):
     wall1 = time.perf_counter()
     if dist is not None:
         dist.barrier()
-    sampler.stop()
     assert pk.pa_get_device_error() == 0
     total_ms = max_over_ranks(total_ms, dist, dev)
     ms_per_step = total_ms / K
@@ -804,10 +952,12 @@ def run_prefill(args, rank, world, dist):
             houts[b].copy_(douts[b], non_blocking=True)
             out_done[b].record(s_out)
     torch.cuda.synchronize()
-    e2e_s = max_over_ranks((time.perf_counter() - p0) / E, dist, dev)
+    wall2 = time.perf_counter()
+    sampler.stop()
+    e2e_s = max_over_ranks((wall2 - p0) / E, dist, dev)
     assert pk.pa_get_device_error() == 0
     if rank != 0:
-        return
+        return None
     flops = prefill_flops(case)
     mma_sync = args.prefill_kernel == "mma_sync"
     att_avg = sum(att_ms) / K
@@ -825,7 +975,7 @@ def run_prefill(args, rank, world, dist):
             if chunked else f"prefill_gqa: {pb} whole prompts, lengths U[16,1024]")
     line = {
         "metric": "paged prefill new tokens/s (append + causal paged attention)", "value": value,
-        "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": desc + "; 32 q / 8 kv heads, head_dim 128, bf16, block_size 16, random "
@@ -846,7 +996,7 @@ def run_prefill(args, rank, world, dist):
                      "algorithmic_flops_per_launch": flops, "avg_launch_ms": att_avg},
         "append_avg_ms": sum(app_ms) / K,
         "gpu_launches": 2 * K,
-        "clocks": sampler.summary(wall0, wall1),
+        "clocks": sampler.summary(wall0, wall2, timed=(wall0, wall1)),
         "e2e": {"value": world * T / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "note": "per step: H2D of q/k/v/slots/tables/lens/query_start from pinned memory, "
@@ -856,13 +1006,13 @@ def run_prefill(args, rank, world, dist):
                        "note": "the same per-step work with a stream sync after every step"},
         "library": os.path.relpath(pk.library_path(), ROOT),
     }
-    if not args.no_cpu_baseline and world == 1:
-        toks, done, el = oracle_prefill_sample(case, args.cpu_seconds)
+    if cpu_seconds is not None and world == 1:
+        toks, done, el = oracle_prefill_sample(case, cpu_seconds)
         line["cpu_baseline"] = {
             "value": toks / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"{done} of {len(case.query_lens)} sequences ({toks} new tokens, random order): oracle "
                       f"append + fp64 causal attention through its own block tables, {el:.1f} s"}
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def main():

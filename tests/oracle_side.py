@@ -8,6 +8,7 @@ path.
 """
 from __future__ import annotations
 
+import time
 from dataclasses import dataclass
 
 import numpy as np
@@ -219,3 +220,26 @@ def prefill_tolerance_ok(got: np.ndarray, ref: np.ndarray):
     err = np.abs(got.astype(np.float64) - ref)
     bar = 1e-2 + BF16_UNIT_ROUNDOFF * np.abs(ref)
     return bool((err <= bar).all()), float(err.max(initial=0.0)), float((err / bar).max(initial=0.0))
+
+
+# ---------------------------------------------------------------------------
+# continuous-batching trace
+# ---------------------------------------------------------------------------
+def oracle_trace_row(trace, layer, step, req, table, length):
+    """Oracle decode output of one request at (layer, step) of a trace: the
+    request's K/V for positions 0..length-1 (generator values) are written
+    through its own block table into a compact pool by the oracle's append,
+    then gathered and attended in fp64. Returns ([H][D] output, seconds of
+    oracle work: append + attention, input generation excluded)."""
+    ids = sorted(set(table))
+    remap = {b: i for i, b in enumerate(ids)}
+    pool = np.zeros((len(ids), 2, trace.num_kv_heads, 16, trace.head_dim), dtype=np.uint16)
+    k, v = trace.kv_values(layer, [req] * length, np.arange(length), "cpu")
+    k, v = storage_bits(k), storage_bits(v)
+    q = storage_bits(trace.q_values(layer, step, [req], "cpu"))
+    slots = [remap[table[p // 16]] * 16 + p % 16 for p in range(length)]
+    tab = [[remap[b] for b in table]]
+    t0 = time.perf_counter()
+    assert oa.reshape_and_cache(pool, k, v, slots) == []
+    out = oa.paged_decode(q, pool, tab, [length], trace.scale, "bf16")[0]
+    return out, time.perf_counter() - t0

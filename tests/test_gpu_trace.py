@@ -19,7 +19,7 @@ from oracle.scheduler import OracleScheduler
 from paged_kv_cache_400_b200 import workloads as wl
 from paged_kv_cache_400_b200.engine import DecodeEngine
 
-from oracle_side import storage_bits
+from oracle_side import oracle_trace_row, storage_bits
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -36,16 +36,7 @@ def layer_inputs(trace, eng, idx, layer, device):
 def oracle_attention(trace, layer, step, req, table, length):
     """Oracle: scatter the request's K/V (generator values) through its own
     block table into a compact pool, then gather-and-attend in fp64."""
-    ids = sorted(set(table))
-    remap = {b: i for i, b in enumerate(ids)}
-    pool = np.zeros((len(ids), 2, trace.num_kv_heads, 16, trace.head_dim), dtype=np.uint16)
-    pos = np.arange(length)
-    k, v = trace.kv_values(layer, [req] * length, pos, "cpu")
-    slots = [remap[table[p // 16]] * 16 + p % 16 for p in range(length)]
-    assert oa.reshape_and_cache(pool, storage_bits(k), storage_bits(v), slots) == []
-    q = storage_bits(trace.q_values(layer, step, [req], "cpu"))
-    tab = [[remap[b] for b in table]]
-    return oa.paged_decode(q, pool, tab, [length], trace.scale, "bf16")[0]
+    return oracle_trace_row(trace, layer, step, req, table, length)[0]
 
 
 def test_trace_with_preemption_matches_oracle():
