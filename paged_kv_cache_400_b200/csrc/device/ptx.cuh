@@ -127,6 +127,33 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Packed fp32 pair arithmetic (sm_100a): two independent round-to-nearest
+// operations in one instruction, each exactly the scalar fmaf / fadd.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 A, B, C;\n\t"
+      "mov.b64 A, {%1, %2};\n\tmov.b64 B, {%3, %4};\n\tmov.b64 C, {%5, %6};\n\t"
+      "fma.rn.f32x2 %0, A, B, C;\n\t}"
+      : "=l"(d)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return make_float2(__uint_as_float((uint32_t)d), __uint_as_float((uint32_t)(d >> 32)));
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 A, B;\n\t"
+      "mov.b64 A, {%1, %2};\n\tmov.b64 B, {%3, %4};\n\t"
+      "add.rn.f32x2 %0, A, B;\n\t}"
+      : "=l"(d)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return make_float2(__uint_as_float((uint32_t)d), __uint_as_float((uint32_t)(d >> 32)));
+}
+// Largest of three (a NaN input is ignored, as by fmaxf).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // bf16 pair in a 32-bit word -> two fp32 (exact widening).
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
