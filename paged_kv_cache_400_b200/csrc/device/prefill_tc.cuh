@@ -10,15 +10,18 @@
 // CTA = (unit of two 128-row query tiles, KV head g, sequence b); a row is
 // (query token, query head of g's group): each tile is 128/G tokens x G heads,
 // so one staged KV tile serves every head of the group and both tiles (twice
-// the MMA work per staged byte). 320 threads in four roles:
+// the MMA work per staged byte). 384 threads in four roles:
 //   warps 0-3, 4-7  softmax, one warp group per query tile: thread r owns row
 //              r of its tile = tensor-memory lane r;
-//   warp 8     producer: both Q tiles by TMA once, then KV tiles of 64 keys
-//              (four 16-token blocks gathered through the table, one TMA box
-//              per block and K|V and head-dim half, the 16 boxes issued by 16
-//              lanes at once) into a 4-stage ring;
-//   warp 9     MMA issuer (one thread): per tile, S = Q K^T into tensor
-//              memory, then O += P V with P read back from tensor memory.
+//   warps 8-9  producers: both Q tiles by TMA once (warp 8), then KV tiles of
+//              64 keys (four 16-token blocks gathered through the table, one
+//              TMA box per block and K|V and head-dim half) into a 4-stage
+//              ring; each warp stages two of the four blocks, its 8 boxes
+//              issued by 8 lanes at once (two warps issue boxes about 1.5x as
+//              fast as one);
+//   warps 10-11 MMA issuers (one thread each), one per query tile: S = Q K^T
+//              into tensor memory, then O += P V with P read back from tensor
+//              memory; the two tiles' MMA chains overlap on the tensor core.
 // Tensor memory (512 columns, so one CTA per SM): per tile t at 256 t, O
 // [0,128) fp32 and two S buffers [128,192), [192,256) fp32, each overwritten in
 // place by its P as packed bf16 pairs. Issue order per tile S_0, S_1, PV_0,
@@ -62,9 +65,10 @@ static_assert(PA_PREFILL_QTILES == 1 || PA_PREFILL_QTILES == 2, "one or two quer
 template <int kQTiles>
 struct TcConfig {
   static constexpr int kStages = kQTiles == 2 ? 4 : 2;
-  static constexpr int kThreads = kQTiles * 128 + 32 + kQTiles * 32;
-  static constexpr int kProducerWarp = kQTiles * 4;
-  static constexpr int kMmaWarp = kQTiles * 4 + 1;  // first of kQTiles issuer warps, one per tile
+  static constexpr int kProducers = 2;              // producer warps, each stages half of every KV tile
+  static constexpr int kThreads = kQTiles * 128 + kProducers * 32 + kQTiles * 32;
+  static constexpr int kProducerWarp = kQTiles * 4;  // first producer warp
+  static constexpr int kMmaWarp = kQTiles * 4 + kProducers;  // first of kQTiles issuer warps, one per tile
   static constexpr uint32_t kTmemCols = kQTiles * 256;
   static constexpr int kSmem = kQTiles * kTcQBytes + kStages * kTcStageBytes + 1024;
 };
@@ -144,8 +148,8 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
     mbar_init(&sh.q_full, 1);
 #pragma unroll
     for (int s = 0; s < S; ++s) {
-      mbar_init(&sh.kv_full[s], 1);
-      mbar_init(&sh.kv_empty[s], kQTiles);  // one release per issuer
+      mbar_init(&sh.kv_full[s], Cfg::kProducers);  // one arrival (with its bytes) per producer warp
+      mbar_init(&sh.kv_empty[s], kQTiles);         // one release per issuer
     }
 #pragma unroll
     for (int t = 0; t < kQTiles; ++t)
@@ -164,6 +168,8 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
     tmem_relinquish();
   }
   if (warp == Cfg::kProducerWarp) {
+    // the first producer warp initialised the barriers: it only arrives (the
+    // second producer warp waits here like the rest)
     __syncwarp();
     named_barrier_arrive(1, Cfg::kThreads);
   } else {
@@ -173,9 +179,10 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
   }
   const uint32_t tmem = sh.tmem_base;  // read by the MMA and softmax warps only
 
-  if (warp == Cfg::kProducerWarp) {
-    // ---- producer ---------------------------------------------------------------
-    if (lane == 0) {
+  if (warp >= Cfg::kProducerWarp && warp < Cfg::kMmaWarp) {
+    // ---- producers: warp pw stages blocks 2 pw, 2 pw + 1 of every 64-key tile --------
+    const int32_t pw = warp - Cfg::kProducerWarp;
+    if (pw == 0 && lane == 0) {
       mbar_arrive_expect_tx(&sh.q_full, kQTiles * kTcQBytes);
 #pragma unroll
       for (int t = 0; t < kQTiles; ++t) {
@@ -210,19 +217,21 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
       // TMA fills whole blocks inside the sequence; the warp writes the
       // sequence's partial last block row by row (rows past L zeroed) and zeros
       // for slots past the last block or with a bad id.
-      int32_t blk[kTcBlocksPerTile];
+      constexpr int32_t kMine = kTcBlocksPerTile / Cfg::kProducers;  // block slots of this warp
+      int32_t blk[kMine];
       uint32_t tma_mask = 0;
 #pragma unroll
-      for (int32_t i = 0; i < kTcBlocksPerTile; ++i) {
+      for (int32_t m = 0; m < kMine; ++m) {
+        const int32_t i = pw * kMine + m;  // block slot in the tile
         const int32_t bi = j * kTcBlocksPerTile + i;
-        blk[i] = __shfl_sync(0xffffffffu, ids, first + i);
-        if (bi < nblocks && (blk[i] < 0 || blk[i] >= p.num_blocks)) {
+        blk[m] = __shfl_sync(0xffffffffu, ids, first + i);
+        if (bi < nblocks && (blk[m] < 0 || blk[m] >= p.num_blocks)) {
           if (lane == 0) raise_device_error(PA_DEVERR_BLOCK);
-          blk[i] = -1;
+          blk[m] = -1;
         }
-        const int32_t rows = (bi < nblocks && blk[i] >= 0) ? min(16, L - bi * 16) : 0;
+        const int32_t rows = (bi < nblocks && blk[m] >= 0) ? min(16, L - bi * 16) : 0;
         if (rows == 16) {
-          tma_mask |= 1u << i;
+          tma_mask |= 1u << m;
           continue;
         }
         // 16 rows x 16 chunks of 16 bytes, K and V: 512 chunks over the warp
@@ -232,12 +241,12 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
           const int32_t c = e & 15;  // 16-byte chunk of the 256-byte row
           uint4 val = make_uint4(0, 0, 0, 0);
           if (row < rows)
-            val = __ldg(pool + ((((size_t)blk[i] * 2 + kv) * p.num_kv_heads + g) * 16 + row) * 16 + c);
+            val = __ldg(pool + ((((size_t)blk[m] * 2 + kv) * p.num_kv_heads + g) * 16 + row) * 16 + c);
           const int32_t key = i * 16 + row;
           *reinterpret_cast<uint4*>(st + tc_region(kv, c >> 3) + key * 128 + (((c & 7) ^ (key & 7)) << 4)) = val;
         }
       }
-      if (tma_mask != (1u << kTcBlocksPerTile) - 1) fence_proxy_async_smem();  // the warp wrote slots
+      if (tma_mask != (1u << kMine) - 1) fence_proxy_async_smem();  // the warp wrote slots
       __syncwarp();
       if (lane == 0) {
         const uint32_t bytes = (uint32_t)__popc(tma_mask) * 4u * 2048u;
@@ -245,12 +254,13 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
         else mbar_arrive(&sh.kv_full[s]);
       }
       __syncwarp();
-      // one TMA box per lane: lane = 4 x block slot + 2 x (K|V) + head-dim half
-      const int32_t my_blk = __shfl_sync(0xffffffffu, ids, first + ((lane >> 2) & 3));
-      if (lane < 4 * kTcBlocksPerTile && ((tma_mask >> (lane >> 2)) & 1u)) {
+      // one TMA box per lane: lane = 4 x (this warp's block m) + 2 x (K|V) + head-dim half
+      const int32_t slot = pw * kMine + ((lane >> 2) & (kMine - 1));
+      const int32_t my_blk = __shfl_sync(0xffffffffu, ids, first + slot);
+      if (lane < 4 * kMine && ((tma_mask >> (lane >> 2)) & 1u)) {
         const int kv = (lane >> 1) & 1;
         const int half = lane & 1;
-        tma_load_5d(st + tc_region(kv, half) + (lane >> 2) * 2048, &pool_map, &sh.kv_full[s], 64 * half, 0, g, kv,
+        tma_load_5d(st + tc_region(kv, half) + slot * 2048, &pool_map, &sh.kv_full[s], 64 * half, 0, g, kv,
                     my_blk);
       }
     }
@@ -340,19 +350,17 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
       tmem_ld64_wait(sbuf, sr);
       const int32_t key0 = j * kTcKeys;
       const bool diag = key0 + kTcKeys - 1 > P;
-      float mt = -INFINITY;  // tile max of the raw scores
       if (diag) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < 64; ++c)
           if (key0 + c > P) sr[c] = __float_as_uint(-INFINITY);
-          mt = fmaxf(mt, __uint_as_float(sr[c]));
-        }
-      } else {
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent chains
-#pragma unroll
-        for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sr[c]));
-        mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
+      // tile max of the raw scores: three-input max, four independent chains
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        m4[c & 3] = max3(m4[c & 3], __uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]));
+      float mt = max3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
       mt *= p.scale_log2;
       if (j == 0) {
         m_ref = mt;  // key 0 is never masked: finite
@@ -380,24 +388,26 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
           }
         }
       }
-      // p = 2^(s * scale - m) on the special-function unit
-      const float neg_m = -m_ref;
+      // p = 2^(s * scale - m) on the special-function unit; the exponent
+      // arguments and the row sum two columns per instruction
+      const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
+      const float2 neg_m2 = make_float2(-m_ref, -m_ref);
       uint32_t pw[32];
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        const float x0 = fmaf(__uint_as_float(sr[2 * c]), p.scale_log2, neg_m);
-        const float x1 = fmaf(__uint_as_float(sr[2 * c + 1]), p.scale_log2, neg_m);
-        float p0 = ex2_sfu(x0);
-        float p1 = ex2_sfu(x1);
+        const float2 x =
+            fma2(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), scale2, neg_m2);
+        float p0 = ex2_sfu(x.x);
+        float p1 = ex2_sfu(x.y);
         if (diag) {  // masked keys contribute exactly 0
           p0 = key0 + 2 * c <= P ? p0 : 0.f;
           p1 = key0 + 2 * c + 1 <= P ? p1 : 0.f;
         }
-        sum4[c & 3] += p0 + p1;
+        sum2[c & 1] = add2(sum2[c & 1], make_float2(p0, p1));
         pw[c] = pack_bf16x2(p0, p1);
       }
-      l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      l += (sum2[0].x + sum2[1].x) + (sum2[0].y + sum2[1].y);
       tmem_st32(sbuf, pw);
       tmem_wait_st();
       tc_fence_before_sync();
