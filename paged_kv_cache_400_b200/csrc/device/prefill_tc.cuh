@@ -25,8 +25,9 @@
 // Tensor memory (512 columns, so one CTA per SM): per tile t at 256 t, O
 // [0,128) fp32 and two S buffers [128,192), [192,256) fp32, each overwritten in
 // place by its P as packed bf16 pairs. Issue order per tile S_0, S_1, PV_0,
-// S_2, PV_1, ..., the two tiles interleaved, so the tensor core works on one
-// tile while the other's softmax runs. The running max is only raised when a
+// S_2, PV_1, ... (S_{j+1} after PV_j instead when its K/V tile is not in yet),
+// the two tiles interleaved, so the tensor core works on one tile while the
+// other's softmax runs. The running max is only raised when a
 // tile's max exceeds it by more than 2^8 (log2 domain), so O in tensor memory
 // is rescaled rarely; O and the row sum l always share the same reference max,
 // so the final O / l is exact up to rounding.
@@ -301,7 +302,16 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
       if (ok && ntt > 0) issue_s(0);
       for (int32_t j = 0; j < nt_max && ok; ++j) {
         if (j < ntt) {
-          if (j + 1 < ntt) issue_s(j + 1);
+          // S_{j+1} goes ahead of PV_j when its K/V tile is already in;
+          // otherwise PV_j is issued as soon as P_j is written and S_{j+1}
+          // follows it, so a late K/V tile does not hold PV_j back
+          bool s_next = false;
+          if (j + 1 < ntt &&
+              (kv_ready >= j + 1 || mbar_test_wait(&sh.kv_full[(j + 1) % S], (uint32_t)((j + 1) / S) & 1u))) {
+            if (kv_ready < j + 1) kv_ready = j + 1;
+            issue_s(j + 1);
+            s_next = true;
+          }
           ok = ok && mbar_wait_bounded(&sh.p_full[t][j & 1], (uint32_t)(j >> 1) & 1u, kWaitLimitNs);
           if (!ok) break;
           tc_fence_after_sync();
@@ -316,6 +326,7 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
                       (j > 0 || kk > 0) ? 1u : 0u);
           tc_commit(&sh.pv_done[t][j & 1]);
           if (j + S < nt_max) tc_commit(&sh.kv_empty[j % S]);
+          if (j + 1 < ntt && !s_next) issue_s(j + 1);
         } else if (j + S < nt_max) {
           // this tile never reads KV tile j; release it in order, after its load
           ensure_kv(j);
