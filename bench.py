@@ -215,7 +215,7 @@ DECODE_KERNEL_SOURCES = ("common.cuh", "decode_common.cuh", "decode_staged.cuh",
 
 
 PREFILL_KERNEL_SOURCES = ("common.cuh", "ptx.cuh", "tcgen05.cuh", "decode_common.cuh", "decode_staged.cuh",
-                          "prefill.cuh", "prefill_tc.cuh")
+                          "prefill_common.cuh", "prefill_tc.cuh")
 
 
 def kernel_source_digest(sources=None):
@@ -969,7 +969,7 @@ def measure_prefill(args, rank, world, dist, chunked, K, warmup, cpu_seconds):
                                   "captured at 64 sequences only")
     if args.prefill_kernel == "tcgen05" and pb == 64:
         traffic, traffic_src = recorded_traffic(
-            os.path.join(ROOT, "profiles", f"prefill_tc_{'chunked' if chunked else 'prompts'}_b64.md"),
+            os.path.join(ROOT, "profiles", f"prefill_tc_{'chunked' if chunked else 'prompts'}_b64.json"),
             PREFILL_KERNEL_SOURCES)
     desc = (f"chunked_prefill_gqa: {pb} sequences, cached context U[0,3072] + a 512-token chunk"
             if chunked else f"prefill_gqa: {pb} whole prompts, lengths U[16,1024]")
