@@ -57,7 +57,7 @@ def parse_args():
                     help="prefix_trace: run without automatic prefix caching (for comparison)")
     ap.add_argument("--prefill", action="store_true",
                     help="trace: also run the admitted prompts' causal prefill attention (pa_prefill) per layer")
-    ap.add_argument("--prefill-kernel", choices=["tcgen05", "tcgen05_1tile", "mma_sync"], default="tcgen05",
+    ap.add_argument("--prefill-kernel", choices=["tcgen05", "mma_sync"], default="tcgen05",
                     help="prefill workloads: the product kernel, or a comparison build's kernel")
     ap.add_argument("--graphs", action="store_true",
                     help="trace: replay each step's decode over all layers as a CUDA graph")
@@ -986,9 +986,7 @@ def measure_prefill(args, rank, world, dist, chunked, K, warmup, cpu_seconds):
                    "l2": "no flush: K/V read %.2f GB per step (> 126 MB L2), q/out %.2f GB"
                          % (kv_bytes / 1e9, 2 * T * case.num_heads * case.head_dim * 2 / 1e9)},
         "roofline": {"kernel": ("prefill_kernel (mma.sync m16n8k16; comparison build)" if mma_sync else
-                                "prefill_tc_kernel (tcgen05.mma, accumulators in tensor memory)"
-                                + ("; one query tile per CTA, comparison build"
-                                   if args.prefill_kernel == "tcgen05_1tile" else "")),
+                                "prefill_tc_kernel (tcgen05.mma, accumulators in tensor memory)"),
                      "bound": "tensor", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": peak_src,
                      "traffic": traffic, "traffic_source": traffic_src,
@@ -1037,8 +1035,7 @@ def main():
             run_trace(args, rank, world)
         elif args.workload in ("prefill", "chunked_prefill"):
             from paged_kv_cache_400_b200 import binding as bd
-            variant = {"tcgen05": None, "tcgen05_1tile": "prefill_1tile",
-                       "mma_sync": "prefill_mma_sync"}[args.prefill_kernel]
+            variant = {"tcgen05": None, "mma_sync": "prefill_mma_sync"}[args.prefill_kernel]
             with bd.use_variant(variant):
                 run_prefill(args, rank, world, dist)
         else:

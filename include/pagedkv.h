@@ -249,13 +249,13 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* kv_pool,
  * PA_DEVERR_SEQLEN and skips sequence b; a block id outside the pool sets
  * PA_DEVERR_BLOCK (that block's contribution is undefined, nothing is read
  * from it). A wait on staged data that exceeds 2 s sets PA_DEVERR_TIMEOUT; while
- * that bit is set (until pa_get_device_error reads it), prefill tiles that
- * start later skip their work. Allocates nothing.
+ * that bit is set (until pa_get_device_error reads it), prefill work units
+ * taken later are skipped. Allocates nothing.
  * Kernel: tcgen05 MMAs with tensor-memory accumulators, two 128-row query
- * tiles per CTA. There is no run-time kernel choice: the mma.sync kernel and a
- * one-tile tcgen05 variant exist only in separate comparison builds of this
- * library (compiled with PA_PREFILL_MMA_SYNC or PA_PREFILL_QTILES=1; same
- * results within rounding).
+ * tiles per work unit, about one persistent CTA per SM taking units in launch
+ * order. There is no run-time kernel choice: the mma.sync kernel exists only
+ * in a separate comparison build of this library (compiled with
+ * PA_PREFILL_MMA_SYNC; same results within rounding).
  */
 pa_status pa_prefill(void* out, const void* q, const void* kv_pool,
                      const int32_t* block_tables, int32_t max_blocks_per_seq,

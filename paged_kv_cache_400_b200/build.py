@@ -9,7 +9,6 @@ Comparison builds (build(variant=...)) compile the same sources with one
 compile-time switch into a library of their own, libpagedkv_<variant>.so; the
 product library never contains their kernels:
   prefill_mma_sync   pa_prefill runs the mma.sync prefill kernel
-  prefill_1tile      pa_prefill's tcgen05 kernel takes one query tile per CTA
 """
 from __future__ import annotations
 
@@ -33,7 +32,6 @@ SOURCES = [
 ]
 VARIANTS = {
     "prefill_mma_sync": ["-DPA_PREFILL_MMA_SYNC"],
-    "prefill_1tile": ["-DPA_PREFILL_QTILES=1"],
 }
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-shared", "-Xcompiler", "-fPIC",

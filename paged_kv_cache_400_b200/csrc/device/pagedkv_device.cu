@@ -1,6 +1,7 @@
 // C-ABI device entry points of libpagedkv.so: argument checks, kernel choice,
 // launches. All kernels live in this one translation unit so they share the
 // per-device error word without relocatable device code.
+#include <algorithm>
 #include <cmath>
 #include <mutex>
 

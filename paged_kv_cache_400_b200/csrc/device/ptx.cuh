@@ -102,6 +102,28 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// 3-D tiled TMA store of one box from shared memory (bulk-group completion:
+// the issuing thread commits the group and waits for its reads before the
+// shared memory is written again or the CTA exits). Coordinates must not be
+// negative.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int32_t c0, int32_t c1,
+                                             int32_t c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(src))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until every bulk group this thread committed has finished reading its
+// shared-memory source.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Waits until every bulk group this thread committed has completed (its
+// global writes performed).
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Named CTA barrier `id` over `count` threads: sync waits for all of them,
 // arrive counts this thread without waiting.
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
@@ -165,6 +187,36 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// ---- cluster launch control (sm_100) -------------------------------------------
+// Asks the hardware scheduler to cancel one CTA of this grid that has not
+// started yet. The 16-byte response is written asynchronously to `resp`
+// (16-byte aligned shared memory) and completes 16 transaction bytes on
+// `bar`, which the caller has armed with mbar_arrive_expect_tx(bar, 16).
+// A CTA sends no further request after a response that reported no CTA.
+__device__ __forceinline__ void clc_try_cancel(void* resp, uint64_t* bar) {
+  asm volatile("clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
+                   smem_addr(resp)),
+               "r"(smem_addr(bar))
+               : "memory");
+}
+// Reads a completed response: true with the x index of the canceled CTA (whose
+// work the caller now owns), false when no CTA was left to cancel.
+__device__ __forceinline__ bool clc_canceled_x(const void* resp, int32_t& x) {
+  uint32_t ok, cx;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b128 r;\n\t"
+      "ld.shared.b128 r, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "mov.u32 %1, 0;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid.v4.b32.b128 {%1, _, _, _}, r;\n\t}"
+      : "=r"(ok), "=r"(cx)
+      : "r"(smem_addr(resp))
+      : "memory");
+  x = (int32_t)cx;
+  return ok != 0;
 }
 
 // bf16 pair in a 32-bit word -> two fp32 (exact widening).

@@ -21,12 +21,11 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-@pytest.fixture(autouse=True, params=["tcgen05", "tcgen05_1tile", "mma_sync"])
+@pytest.fixture(autouse=True, params=["tcgen05", "mma_sync"])
 def prefill_kernel(request):
     """Every test runs on each prefill kernel: the product library's tcgen05
-    kernel, and the two comparison builds (tcgen05 with one query tile per
-    CTA, and the mma.sync kernel), each a library of its own."""
-    variant = {"tcgen05": None, "tcgen05_1tile": "prefill_1tile", "mma_sync": "prefill_mma_sync"}[request.param]
+    kernel and the comparison build's mma.sync kernel (a library of its own)."""
+    variant = {"tcgen05": None, "mma_sync": "prefill_mma_sync"}[request.param]
     with bd.use_variant(variant):
         yield request.param
 
@@ -93,6 +92,48 @@ def test_empty_sequences_mixed():
     ref, _ = oracle_prefill_all(case, ost)
     ok, err, _ = prefill_tolerance_ok(out.float().cpu().numpy(), ref)
     assert ok, err
+
+
+def test_many_sequences_ragged():
+    # 75 sequences (three passes of the kernel's 32-sequence unit lookup),
+    # zero-length ones among them, chunks across tile and block boundaries
+    rng = np.random.default_rng(14)
+    n = rng.integers(0, 140, size=75)
+    n[[0, 31, 32, 33, 63, 74]] = [0, 0, 65, 1, 0, 129]
+    ctx = rng.integers(0, 90, size=75)
+    case = wl.prefill_custom("many", 14, ctx.tolist(), n.tolist(), 16, 4)
+    check_full(case)
+
+
+@pytest.mark.parametrize("where", [1, 40])
+def test_malformed_query_ranges_flagged(where):
+    # a decreasing query_start (n < 0) or a range past the last q row makes
+    # the sequence count no work and sets PA_DEVERR_SEQLEN, also when it comes
+    # after the first 32 sequences; the sequences before it are unaffected
+    lens = [20] * 48
+    case = wl.prefill_custom("badq", 15, [0] * 48, lens, 32, 8)
+    prep = prepare_prefill_step(case)
+    pool = case.make_pool(DEV)
+    k, v = case.make_kv_new(DEV)
+    pk.pa_reshape_and_cache(k, v, pool, torch.from_numpy(prep.slot_mapping).to(DEV))
+    q = case.make_q(DEV)
+    bt = torch.from_numpy(prep.block_tables).to(DEV)
+    sl = torch.from_numpy(prep.seq_lens).to(DEV)
+    ost = oracle_prefill_indices(case)
+    ref = oracle_prefill_rows(case, ost, [(0, 0), (0, 19), (where - 1, 0), (where - 1, 19)])
+    for bad in ("decreasing", "past_end"):
+        qs = prep.query_start.copy()
+        if bad == "decreasing":
+            qs[where + 1] = qs[where] - 5
+        else:
+            qs[where + 1:] = case.num_tokens + 7
+        out = torch.zeros_like(q)
+        pk.pa_prefill(out, q, pool, bt, sl, torch.from_numpy(qs).to(DEV), case.scale, case.max_query_len)
+        torch.cuda.synchronize()
+        assert pk.pa_get_device_error() == pk.PA_DEVERR_SEQLEN, bad
+        rows = [0, 19, int(qs[where - 1]), int(qs[where - 1]) + 19]
+        ok, err, _ = prefill_tolerance_ok(out[rows].float().cpu().numpy(), ref)
+        assert ok, (bad, err)
 
 
 def test_nothing_to_do():
