@@ -70,20 +70,21 @@ constexpr int kTcQBytes = 128 * 256;              // one 128-row query tile x 12
 constexpr float kTcRescaleLog2 = 8.0f;            // raise the reference max past this growth
 
 // Two query tiles of 128 rows share every staged KV tile: one CTA per SM (all
-// 512 tensor-memory columns, 225 KB of shared memory), a 3-deep KV ring.
+// 512 tensor-memory columns, 225 KB of shared memory), a 4-deep KV ring.
 template <int kQTiles>
 struct TcConfig {
-  static constexpr int kStages = 3;
+  static constexpr int kStages = 4;
   static constexpr int kProducers = 2;              // producer warps, each stages half of every KV tile
   static constexpr int kSoftmaxWarps = kQTiles * 4;
-  static constexpr int kThreads = kQTiles * 128 + kProducers * 32 + kQTiles * 32;
-  static constexpr int kProducerWarp = kQTiles * 4;  // first producer warp (the scheduler)
+  static constexpr int kProducerWarp = kQTiles * 4;          // first producer warp
   static constexpr int kMmaWarp = kQTiles * 4 + kProducers;  // first of kQTiles issuer warps, one per tile
+  static constexpr int kSchedWarp = kMmaWarp + kQTiles;      // the scheduler
+  static constexpr int kThreads = (kSchedWarp + 1) * 32;
   static constexpr uint32_t kTmemCols = kQTiles * 256;
-  // readers of each published unit: the second producer warp, the issuers, the softmax warps
-  static constexpr uint32_t kUnitReaders = (kProducers - 1) + kQTiles + kSoftmaxWarps;
-  // Q tiles, the K/V ring, one output staging tile per query tile, alignment slack
-  static constexpr int kSmem = kQTiles * kTcQBytes + kStages * kTcStageBytes + kQTiles * kTcQBytes + 1024;
+  // readers of each published unit: the producers, the issuers, the softmax warps
+  static constexpr uint32_t kUnitReaders = kProducers + kQTiles + kSoftmaxWarps;
+  // Q tiles, the K/V ring, half an output tile of staging per query tile, alignment slack
+  static constexpr int kSmem = kQTiles * kTcQBytes + kStages * kTcStageBytes + kQTiles * (kTcQBytes / 2) + 1024;
 };
 constexpr int kTcQTiles = 2;
 
@@ -99,6 +100,7 @@ struct PrefillTcShared {
   uint64_t clc_bar;              // cancellation response written
   uint64_t unit_full[2];         // unit slot published
   uint64_t unit_empty[2];        // unit slot read by every reader
+  uint64_t unit_taken;           // the producers have taken the latest unit (one arrival per producer warp)
   uint64_t q_full;               // both Q tiles of the current unit loaded
   uint64_t q_empty;              // every S MMA of the current unit complete (one commit per issuer)
   uint64_t kv_full[kStages];
@@ -106,8 +108,8 @@ struct PrefillTcShared {
   uint64_t s_full[kQTiles][2];   // S of tile t's KV step J ready: s_full[t][J & 1]
   uint64_t p_full[kQTiles][2];   // P of step J written (one arrival per softmax warp)
   uint64_t pv_done[kQTiles][2];  // PV of step J complete: pv_done[t][J & 1]
-  uint64_t stage_free[kQTiles];  // tile t's previous output store has read its staging buffer
-  uint64_t staged[kQTiles];      // tile t's rows written to staging (one arrival per softmax warp)
+  uint64_t stage_free[kQTiles];  // tile t's previous output store has read its staging half
+  uint64_t staged[kQTiles];      // tile t's half rows written to staging (one arrival per softmax warp)
   uint32_t tmem_base;
 };
 
@@ -219,13 +221,14 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
   const int32_t warp = threadIdx.x >> 5;
   const int32_t lane = threadIdx.x & 31;
 
-  if (warp == Cfg::kProducerWarp && lane == 0) {
+  if (warp == Cfg::kSchedWarp && lane == 0) {
     mbar_init(&sh.clc_bar, 1);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.unit_full[i], 1);
       mbar_init(&sh.unit_empty[i], Cfg::kUnitReaders);
     }
+    mbar_init(&sh.unit_taken, Cfg::kProducers);
     mbar_init(&sh.q_full, 1);
     mbar_init(&sh.q_empty, kQTiles);  // one commit (or arrival) per issuer
 #pragma unroll
@@ -275,11 +278,7 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
 
   if (warp >= Cfg::kProducerWarp && warp < Cfg::kMmaWarp) {
     // ---- producers: warp pw stages blocks 2 pw, 2 pw + 1 of every 64-key tile -------
-    // Warp 0 of the two also schedules: it resolves its CTA's own unit, then
-    // cancels not-yet-started CTAs and takes their units, publishing each to
-    // the other roles through a two-slot ring, and loads its Q tiles.
     const int32_t pw = warp - Cfg::kProducerWarp;
-    const bool scheduler = pw == 0;
 
     // stages the unit's KV tiles (global tile index jkv0 + j) into the ring
     auto stream_kv = [&](const TcUnit& u, uint32_t jkv0) -> bool {
@@ -368,130 +367,120 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
     uint32_t k = 0;    // units taken
     uint32_t jkv = 0;  // KV tiles staged (both producer warps count alike)
     bool ok = true;
-    if (scheduler) {
-      // the unit at CTA index i, unless i lies past the last unit, its
-      // sequence is malformed, or a wait has timed out somewhere in the grid
-      // (then the remaining units are skipped; the error stays set until the
-      // host reads it)
-      auto resolve = [&](int32_t i, TcUnit& u) -> bool {
-        if (!find_unit(p, num_seqs, U, i, u)) return false;
-        if (u.L < u.n || (int64_t)u.L > (int64_t)p.max_blocks * 16) {
-          if (u.unit == 0 && u.g == 0 && lane == 0) raise_device_error(PA_DEVERR_SEQLEN);
-          return false;
-        }
-        return !(*reinterpret_cast<volatile unsigned int*>(&g_error_word) & PA_DEVERR_TIMEOUT);
-      };
-      auto request = [&]() {
+    for (;;) {
+      TcUnit u;
+      if (!__all_sync(0xffffffffu, read_unit(k, u))) {
+        ok = false;
+        break;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&sh.unit_empty[k & 1]);
+        if (u.n >= 0) mbar_arrive(&sh.unit_taken);
+      }
+      if (u.n < 0) break;
+      ok = stream_kv(u, jkv);
+      int32_t nt[kQTiles], nb;
+      jkv += (uint32_t)unit_tiles<kQTiles>(u, QT, nt, nb);
+      ++k;
+      if (!ok) break;
+    }
+    // the asynchronous releases still owed to the ring land before the CTA exits
+    if (ok && pw == 0)
+      for (uint32_t J = jkv > (uint32_t)S ? jkv - S : 0; J < jkv && ok; ++J)
+        ok = mbar_wait_bounded(&sh.kv_empty[J % S], (J / S) & 1u, kWaitLimitNs);
+    if (!__all_sync(0xffffffffu, ok) && lane == 0) raise_device_error(PA_DEVERR_TIMEOUT);
+  } else if (warp == Cfg::kSchedWarp) {
+    // ---- scheduler: resolves the CTA's own unit, then cancels not-yet-started
+    // CTAs and takes their units, publishing each to the other roles through a
+    // two-slot ring, and loads each unit's Q tiles once the previous unit's S
+    // MMAs have completed. The next unit is requested once the producers have
+    // taken the last one, so the CTA holds at most one unit beyond the one in
+    // its K/V ring.
+    // The unit at CTA index i, unless i lies past the last unit, its sequence
+    // is malformed, or a wait has timed out somewhere in the grid (then the
+    // remaining units are skipped; the error stays set until the host reads it).
+    auto resolve = [&](int32_t i, TcUnit& u) -> bool {
+      if (!find_unit(p, num_seqs, U, i, u)) return false;
+      if (u.L < u.n || (int64_t)u.L > (int64_t)p.max_blocks * 16) {
+        if (u.unit == 0 && u.g == 0 && lane == 0) raise_device_error(PA_DEVERR_SEQLEN);
+        return false;
+      }
+      return !(*reinterpret_cast<volatile unsigned int*>(&g_error_word) & PA_DEVERR_TIMEOUT);
+    };
+    bool ok = true;
+    bool can_cancel = true;  // no request has come back empty yet
+    uint32_t clc_phase = 0;
+    // one cancellation request; false once none is left (or on a timeout)
+    auto take_next = [&](TcUnit& u) -> bool {
+      while (can_cancel && ok) {
         if (lane == 0) {
           mbar_arrive_expect_tx(&sh.clc_bar, 16);
           clc_try_cancel(&sh.clc_resp, &sh.clc_bar);
         }
-      };
-      TcUnit u;
-      bool have = resolve((int32_t)blockIdx.x, u);
-      bool can_cancel = true;  // no request has come back empty yet
-      uint32_t clc_phase = 0;
-      for (;;) {
-        bool asked = false;
-        if (have) {
-          // publish unit k once every reader has taken unit k - 2 from its slot
-          if (k >= 2) ok = mbar_wait_bounded(&sh.unit_empty[k & 1], ((k >> 1) - 1) & 1u, kWaitLimitNs);
-          if (!__all_sync(0xffffffffu, ok)) {
-            ok = false;
-            break;
-          }
-          if (lane == 0) {
-            int32_t* d = sh.unit_desc[k & 1];
-            d[0] = u.b;
-            d[1] = u.g;
-            d[2] = u.unit;
-            d[3] = u.q0;
-            d[4] = u.n;
-            d[5] = u.L;
-            mbar_arrive(&sh.unit_full[k & 1]);
-          }
-          // both Q tiles, once every S MMA of unit k - 1 has completed
-          if (k >= 1) ok = mbar_wait_bounded(&sh.q_empty, (k - 1) & 1u, kWaitLimitNs);
-          if (!__all_sync(0xffffffffu, ok)) {
-            ok = false;
-            break;
-          }
-          if (lane == 0) {
-            const int32_t row = u.q0 + u.unit * U;
-            mbar_arrive_expect_tx(&sh.q_full, kQTiles * kTcQBytes);
-#pragma unroll
-            for (int t = 0; t < kQTiles; ++t) {
-              tma_load_3d(q_smem + t * kTcQBytes, &q_map, &sh.q_full, 0, u.g * G, row + t * QT);
-              tma_load_3d(q_smem + t * kTcQBytes + kTcQBytes / 2, &q_map, &sh.q_full, 64, u.g * G, row + t * QT);
-            }
-          }
-          // ask for the next unit now: the answer is read after this unit's K/V
-          if (can_cancel) {
-            request();
-            asked = true;
-          }
-          ok = stream_kv(u, jkv);
-          int32_t nt[kQTiles], nb;
-          jkv += (uint32_t)unit_tiles<kQTiles>(u, QT, nt, nb);
-          ++k;
-        } else if (can_cancel) {
-          request();
-          asked = true;
-        } else {
+        // the response lands before anything else happens here
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sh.clc_bar, clc_phase, kWaitLimitNs));
+        clc_phase ^= 1u;
+        if (!ok) break;
+        int32_t x = 0;
+        const bool got = clc_canceled_x(&sh.clc_resp, x);
+        fence_proxy_async_smem();  // this read before the next response's write
+        __syncwarp();
+        if (!got) {
+          can_cancel = false;
           break;
         }
-        if (asked) {
-          // a request's response must land before this CTA stops
-          const bool arrived = __all_sync(0xffffffffu, mbar_wait_bounded(&sh.clc_bar, clc_phase, kWaitLimitNs));
-          clc_phase ^= 1u;
-          if (!arrived) {
-            ok = false;
-            break;
-          }
-          int32_t x = 0;
-          const bool got = clc_canceled_x(&sh.clc_resp, x);
-          fence_proxy_async_smem();  // this read before the next response's write
-          __syncwarp();
-          if (got) {
-            have = ok && resolve(x, u);
-          } else {
-            can_cancel = false;
-            have = false;
-          }
-        }
-        if (!ok) break;
+        if (resolve(x, u)) return true;
       }
-      // the end: an empty unit in the next slot stops every reader
-      bool fin = true;
-      if (k >= 2) fin = mbar_wait_bounded(&sh.unit_empty[k & 1], ((k >> 1) - 1) & 1u, kWaitLimitNs);
-      if (__all_sync(0xffffffffu, fin) && lane == 0) {
-        sh.unit_desc[k & 1][4] = -1;
+      return false;
+    };
+    TcUnit u;
+    bool have = resolve((int32_t)blockIdx.x, u) || take_next(u);
+    uint32_t k = 0;  // units published
+    while (have && ok) {
+      // unit k goes into slot k & 1 once every reader has taken unit k - 2
+      if (k >= 2) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sh.unit_empty[k & 1], ((k >> 1) - 1) & 1u,
+                                                                 kWaitLimitNs));
+      if (!ok) break;
+      if (lane == 0) {
+        int32_t* d = sh.unit_desc[k & 1];
+        d[0] = u.b;
+        d[1] = u.g;
+        d[2] = u.unit;
+        d[3] = u.q0;
+        d[4] = u.n;
+        d[5] = u.L;
         mbar_arrive(&sh.unit_full[k & 1]);
       }
-      // the asynchronous arrivals still owed to this CTA's barriers land
-      // before it exits: the last unit's Q release, the last K/V releases
-      if (ok && k >= 1) ok = mbar_wait_bounded(&sh.q_empty, (k - 1) & 1u, kWaitLimitNs);
-      for (uint32_t J = jkv > (uint32_t)S ? jkv - S : 0; J < jkv && ok; ++J)
-        ok = mbar_wait_bounded(&sh.kv_empty[J % S], (J / S) & 1u, kWaitLimitNs);
-      if (!__all_sync(0xffffffffu, ok) && lane == 0) raise_device_error(PA_DEVERR_TIMEOUT);
-    } else {
-      for (;;) {
-        TcUnit u;
-        if (!__all_sync(0xffffffffu, read_unit(k, u))) {
-          ok = false;
-          break;
+      // its Q tiles, once every S MMA of unit k - 1 has completed
+      if (k >= 1) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sh.q_empty, (k - 1) & 1u, kWaitLimitNs));
+      if (!ok) break;
+      if (lane == 0) {
+        const int32_t row = u.q0 + u.unit * U;
+        mbar_arrive_expect_tx(&sh.q_full, kQTiles * kTcQBytes);
+#pragma unroll
+        for (int t = 0; t < kQTiles; ++t) {
+          tma_load_3d(q_smem + t * kTcQBytes, &q_map, &sh.q_full, 0, u.g * G, row + t * QT);
+          tma_load_3d(q_smem + t * kTcQBytes + kTcQBytes / 2, &q_map, &sh.q_full, 64, u.g * G, row + t * QT);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.unit_empty[k & 1]);
-        if (u.n < 0) break;
-        ok = stream_kv(u, jkv);
-        int32_t nt[kQTiles], nb;
-        jkv += (uint32_t)unit_tiles<kQTiles>(u, QT, nt, nb);
-        ++k;
-        if (!ok) break;
       }
-      if (!ok && lane == 0) raise_device_error(PA_DEVERR_TIMEOUT);
+      ++k;
+      // the next unit once the producers have taken this one
+      if (!can_cancel) break;
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sh.unit_taken, (k - 1) & 1u, kWaitLimitNs));
+      if (!ok) break;
+      have = take_next(u);
     }
+    // the end: an empty unit in the next slot stops every reader
+    bool fin = true;
+    if (k >= 2) fin = mbar_wait_bounded(&sh.unit_empty[k & 1], ((k >> 1) - 1) & 1u, kWaitLimitNs);
+    if (__all_sync(0xffffffffu, fin) && lane == 0) {
+      sh.unit_desc[k & 1][4] = -1;
+      mbar_arrive(&sh.unit_full[k & 1]);
+    }
+    // the last unit's Q release (a commit) lands before the CTA exits
+    if (ok && k >= 1) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sh.q_empty, (k - 1) & 1u, kWaitLimitNs));
+    if (!ok && lane == 0) raise_device_error(PA_DEVERR_TIMEOUT);
   } else if (warp >= Cfg::kMmaWarp) {
     // ---- MMA issuers: warp kMmaWarp + t, one thread, drives query tile t -------------
     const int t = warp - Cfg::kMmaWarp;
@@ -594,11 +583,11 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
     const int32_t t = warp >> 2;
     const int32_t r = threadIdx.x - 128 * t;
     const uint32_t lane_base = tmem + t * 256 + ((uint32_t)((warp & 3) * 32) << 16);
-    uint8_t* stage = out_smem + t * kTcQBytes;  // this tile's output rows, in the Q tile layout
+    uint8_t* stage = out_smem + t * (kTcQBytes / 2);  // half of this tile's output rows, in the Q tile layout
     const bool leader = r == 0;                 // issues the tile's output stores
     uint32_t k = 0;   // units taken
     uint32_t js = 0;  // this tile's KV steps of the earlier units
-    uint32_t ne = 0;  // this tile's output epilogues so far
+    uint32_t ne = 0;  // this tile's staged output halves so far
     bool ok = true;
     for (;;) {
       TcUnit u;
@@ -702,68 +691,60 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
         ok = !__any_sync(0xffffffffu, !done);
         if (ok) {
           tc_fence_after_sync();
-          // the tile's previous output store has read the staging buffer
-          // (mbarriers rather than named barriers between the group's warps,
-          // so that every wait is bounded)
-          if (leader) {
-            bulk_wait_group_read0();
-            mbar_arrive(&sh.stage_free[t]);
-          }
-          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sh.stage_free[t], ne & 1u, kWaitLimitNs));
-        }
-        if (ok) {
-          // row r of O / l as bf16 into the staging tile: 128-byte half rows,
-          // 16-byte chunks XOR-swizzled by row (the 128-byte TMA swizzle, which
-          // also spreads a warp's writes over all banks)
+          // O / l as bf16, one head-dim half at a time through the tile's
+          // 16 KB staging half (the Q tile layout: 128-byte rows, 16-byte
+          // chunks XOR-swizzled by row, which also spreads a warp's writes
+          // over all banks). A whole tile leaves by one TMA store per half
+          // that drains while the warps go on; the sequence's last, partial
+          // tile (its rows after the new tokens belong to the next sequence)
+          // by plain stores, each warp its own valid rows. The warps of the
+          // group meet on mbarriers, so that every wait is bounded.
           const float inv = 1.f / l;
-#pragma unroll 1
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t o[32];
-            tmem_ld32_wait(lane_base + 32 * cc, o);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
-              w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
-              w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
-              w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
-              const int32_t chunk = 4 * cc + v;  // dims 8 chunk .. 8 chunk + 7
-              *reinterpret_cast<uint4*>(stage + (chunk >> 3) * (kTcQBytes / 2) + r * 128 +
-                                        (((chunk & 7) ^ (r & 7)) << 4)) = w;
-            }
-          }
-          fence_proxy_async_smem();  // the staging writes before the TMA store reads them
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh.staged[t]);
           const bool whole = te == tb + QT;
-          if (leader) {
-            ok = mbar_wait_bounded(&sh.staged[t], ne & 1u, kWaitLimitNs);
-            if (ok && whole) {
-              // a whole tile: one TMA store per head-dim half; the warps go on
-              // while it drains
-              tma_store_3d(&out_map, stage, 0, u.g * G, u.q0 + tb);
-              tma_store_3d(&out_map, stage + kTcQBytes / 2, 64, u.g * G, u.q0 + tb);
-              bulk_commit_group();
+          const int32_t row0 = (warp & 3) * 32;
+          uint4* out4 = reinterpret_cast<uint4*>(p.out);
+#pragma unroll 1
+          for (int half = 0; half < 2 && ok; ++half) {
+            uint32_t o[64];
+            tmem_ld64_wait(lane_base + 64 * half, o);
+            // the tile's previous store has read the staging half
+            if (leader) {
+              bulk_wait_group_read0();
+              mbar_arrive(&sh.stage_free[t]);
             }
-          }
-          ok = __all_sync(0xffffffffu, ok);
-          ++ne;
-          if (ok && !whole) {
-            // the sequence's last, partial tile (the rows after its new tokens
-            // belong to the next sequence): each warp stores its own valid
-            // rows, four 128-byte half rows per instruction
-            const int32_t row0 = (warp & 3) * 32;
-            uint4* out4 = reinterpret_cast<uint4*>(p.out);
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(&sh.stage_free[t], ne & 1u, kWaitLimitNs));
+            if (!ok) break;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {  // dims 64 half + 8 c .. + 7
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
+              *reinterpret_cast<uint4*>(stage + r * 128 + ((c ^ (r & 7)) << 4)) = w;
+            }
+            fence_proxy_async_smem();  // the staging writes before the TMA store reads them
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.staged[t]);
+            if (leader) {
+              ok = mbar_wait_bounded(&sh.staged[t], ne & 1u, kWaitLimitNs);
+              if (ok && whole) {
+                tma_store_3d(&out_map, stage, 64 * half, u.g * G, u.q0 + tb);
+                bulk_commit_group();
+              }
+            }
+            ok = __all_sync(0xffffffffu, ok);
+            ++ne;
+            if (ok && !whole) {
 #pragma unroll 4
-            for (int i = 0; i < 16; ++i) {
-              const int32_t hr = 4 * i + (lane >> 3);
-              const int32_t rr = row0 + (hr >> 1);
-              const int32_t half = hr & 1;
-              const int32_t c = lane & 7;
-              const int32_t tk = tb + rr / G;
-              if (tk < te)
-                out4[((size_t)(u.q0 + tk) * p.num_heads + (size_t)u.g * G + rr % G) * 16 + half * 8 + c] =
-                    *reinterpret_cast<const uint4*>(stage + half * (kTcQBytes / 2) + rr * 128 + ((c ^ (rr & 7)) << 4));
+              for (int i = 0; i < 8; ++i) {  // four 128-byte half rows per instruction
+                const int32_t rr = row0 + 4 * i + (lane >> 3);
+                const int32_t c = lane & 7;
+                const int32_t tk = tb + rr / G;
+                if (tk < te)
+                  out4[((size_t)(u.q0 + tk) * p.num_heads + (size_t)u.g * G + rr % G) * 16 + half * 8 + c] =
+                      *reinterpret_cast<const uint4*>(stage + rr * 128 + ((c ^ (rr & 7)) << 4));
+              }
             }
           }
         }
