@@ -185,6 +185,93 @@ __device__ __forceinline__ bool find_unit(const PrefillParams& p, int32_t num_se
   return found;
 }
 
+// Up to this many sequences the units go out longest sequence first (see
+// UnitOrder); beyond it in sequence order.
+constexpr int kTcSortedSeqs = 128;
+
+// The launch order of the units when the sequences are sorted by KV length L,
+// longest first (ties by index): every sequence's units (all KV heads
+// together, each head's units last-first) stay contiguous, sequence s's from
+// index start[s / 32] on, cnt[s / 32] of them, held by lane s % 32. The
+// longest units start first and the grid ends on short ones, so the SMs run
+// out of work at nearly the same time. Built once per CTA by its scheduler
+// warp, O(num_seqs^2 / 32) per lane; sequences whose query range is
+// malformed count no units and set PA_DEVERR_SEQLEN.
+struct UnitOrder {
+  int32_t start[kTcSortedSeqs / 32];
+  int32_t cnt[kTcSortedSeqs / 32];
+};
+
+__device__ __forceinline__ void build_unit_order(const PrefillParams& p, int32_t num_seqs, int32_t U,
+                                                 UnitOrder& o) {
+  constexpr int P = kTcSortedSeqs / 32;
+  const int32_t lane = threadIdx.x & 31;
+  int32_t L[P];
+  bool any_bad = false;
+#pragma unroll
+  for (int pp = 0; pp < P; ++pp) {
+    const int32_t s = pp * 32 + lane;
+    L[pp] = -1;
+    o.cnt[pp] = 0;
+    o.start[pp] = 0;
+    if (s < num_seqs) {
+      const int32_t a = __ldg(p.query_start + s);
+      const int32_t n = __ldg(p.query_start + s + 1) - a;
+      const bool bad = a < 0 || n < 0 || n > p.max_query_len || a + n > p.num_tokens;
+      any_bad |= bad;
+      L[pp] = __ldg(p.seq_lens + s);
+      o.cnt[pp] = bad ? 0 : (n + U - 1) / U * p.num_kv_heads;
+    }
+  }
+  // start of s = the units of every sequence ahead of it: longer, or as long
+  // with a lower index
+#pragma unroll
+  for (int qq = 0; qq < P; ++qq) {
+    if (qq * 32 >= num_seqs) break;
+#pragma unroll 4
+    for (int src = 0; src < 32; ++src) {
+      const int32_t Lo = __shfl_sync(0xffffffffu, L[qq], src);
+      const int32_t co = __shfl_sync(0xffffffffu, o.cnt[qq], src);
+      const int32_t so = qq * 32 + src;
+#pragma unroll
+      for (int pp = 0; pp < P; ++pp) {
+        const int32_t s = pp * 32 + lane;
+        if (Lo > L[pp] || (Lo == L[pp] && so < s)) o.start[pp] += co;
+      }
+    }
+  }
+  if (__any_sync(0xffffffffu, any_bad) && lane == 0) raise_device_error(PA_DEVERR_SEQLEN);
+}
+
+// Unit idx of a UnitOrder (the calling warp); false past the last unit.
+__device__ __forceinline__ bool find_unit_sorted(const PrefillParams& p, const UnitOrder& o, int32_t idx,
+                                                 TcUnit& u) {
+  constexpr int P = kTcSortedSeqs / 32;
+  int32_t seq = -1, st = 0, ct = 0;
+#pragma unroll
+  for (int pp = 0; pp < P; ++pp) {
+    const uint32_t hit = __ballot_sync(0xffffffffu, idx >= o.start[pp] && idx < o.start[pp] + o.cnt[pp]);
+    const int32_t src = hit ? __ffs(hit) - 1 : 0;
+    const int32_t st_pp = __shfl_sync(0xffffffffu, o.start[pp], src);
+    const int32_t ct_pp = __shfl_sync(0xffffffffu, o.cnt[pp], src);
+    if (hit && seq < 0) {
+      seq = pp * 32 + src;
+      st = st_pp;
+      ct = ct_pp;
+    }
+  }
+  if (seq < 0) return false;
+  const int32_t local = idx - st;
+  const int32_t units = ct / p.num_kv_heads;
+  u.b = seq;
+  u.g = local / units;
+  u.unit = units - 1 - local % units;
+  u.q0 = __ldg(p.query_start + seq);
+  u.n = __ldg(p.query_start + seq + 1) - u.q0;
+  u.L = __ldg(p.seq_lens + seq);
+  return true;
+}
+
 // KV tiles of a unit: returns the unit's count (its last query tile's) and
 // sets nt[t] for each query tile (0 for a tile past the sequence's new tokens).
 template <int kQTiles>
@@ -400,8 +487,11 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
     // The unit at CTA index i, unless i lies past the last unit, its sequence
     // is malformed, or a wait has timed out somewhere in the grid (then the
     // remaining units are skipped; the error stays set until the host reads it).
+    UnitOrder order;
+    const bool sorted = num_seqs <= kTcSortedSeqs;
+    if (sorted) build_unit_order(p, num_seqs, U, order);
     auto resolve = [&](int32_t i, TcUnit& u) -> bool {
-      if (!find_unit(p, num_seqs, U, i, u)) return false;
+      if (!(sorted ? find_unit_sorted(p, order, i, u) : find_unit(p, num_seqs, U, i, u))) return false;
       if (u.L < u.n || (int64_t)u.L > (int64_t)p.max_blocks * 16) {
         if (u.unit == 0 && u.g == 0 && lane == 0) raise_device_error(PA_DEVERR_SEQLEN);
         return false;

@@ -105,13 +105,27 @@ def test_many_sequences_ragged():
     check_full(case)
 
 
-@pytest.mark.parametrize("where", [1, 40])
+def test_more_sequences_than_the_sorted_order():
+    # 150 sequences: past 128 the units go out in sequence order (the lookup
+    # by prefix sum over passes of 32); equal lengths among them (ties)
+    rng = np.random.default_rng(16)
+    n = rng.integers(0, 70, size=150)
+    n[[0, 64, 127, 128, 149]] = [0, 33, 0, 65, 1]
+    ctx = rng.integers(0, 40, size=150)
+    ctx[100:110] = 7
+    n[100:110] = 20
+    case = wl.prefill_custom("many150", 16, ctx.tolist(), n.tolist(), 16, 8)
+    check_full(case)
+
+
+@pytest.mark.parametrize("where", [1, 40, 140])
 def test_malformed_query_ranges_flagged(where):
     # a decreasing query_start (n < 0) or a range past the last q row makes
     # the sequence count no work and sets PA_DEVERR_SEQLEN, also when it comes
-    # after the first 32 sequences; the sequences before it are unaffected
-    lens = [20] * 48
-    case = wl.prefill_custom("badq", 15, [0] * 48, lens, 32, 8)
+    # after the first 32 sequences or past the sorted order's 128; the
+    # sequences before it are unaffected
+    lens = [20] * 150
+    case = wl.prefill_custom("badq", 15, [0] * 150, lens, 32, 8)
     prep = prepare_prefill_step(case)
     pool = case.make_pool(DEV)
     k, v = case.make_kv_new(DEV)
