@@ -14,27 +14,29 @@
 //
 // Persistent CTAs: the grid has one CTA per unit, but a running CTA takes the
 // next units itself by cancelling CTAs that have not started (cluster launch
-// control), so about one CTA per SM runs and one unit's start (Q and first
-// K/V loads, first S) and end (last PV, output stores) overlap its neighbours'
-// work instead of leaving the SM idle between CTAs. The unit order is the
-// launch order, and the hardware balances it as it would balance CTAs.
+// control), so about one CTA per SM runs, set up once, and one unit's start
+// (Q and first K/V loads, first S) and end (last PV, output stores) overlap
+// its neighbours' work instead of leaving the SM idle between CTAs. Units go
+// out longest sequence first, so the grid ends on short ones.
 //
-// 384 threads in four roles:
+// 416 threads in five roles:
 //   warps 0-3, 4-7  softmax, one warp group per query tile: thread r owns row
 //              r of its tile = tensor-memory lane r; at the end of a unit they
-//              write the normalised rows into the tile's staging buffer, which
-//              one TMA store copies out (plain stores for a sequence's last,
-//              partial tile) while the warps go on with the next unit;
-//   warps 8-9  producers: warp 8 also schedules (takes the next unit,
-//              publishes it to the other roles, loads both Q tiles by TMA);
-//              both stream the K/V tiles of 64 keys (four 16-token blocks
-//              gathered through the table, one TMA box per block and K|V and
-//              head-dim half) into a 3-stage ring that runs on across units,
-//              each warp staging two of the four blocks (two warps issue
-//              boxes about 1.5x as fast as one);
+//              stage the normalised rows one head-dim half at a time, and one
+//              TMA store per half copies a whole tile out while the warps go
+//              on (plain stores for a sequence's last, partial tile);
+//   warps 8-9  producers: stream the K/V tiles of 64 keys (four 16-token
+//              blocks gathered through the table, one TMA box per block and
+//              K|V and head-dim half) into a 4-stage ring that runs on across
+//              units, each warp staging two of the four blocks (two warps
+//              issue boxes about 1.5x as fast as one);
 //   warps 10-11 MMA issuers (one thread each), one per query tile: S = Q K^T
 //              into tensor memory, then O += P V with P read back from tensor
-//              memory; the two tiles' MMA chains overlap on the tensor core.
+//              memory; the two tiles' MMA chains overlap on the tensor core;
+//   warp 12    scheduler: takes the units (its own, then cancelled CTAs'),
+//              publishes each to the other roles through a two-slot ring and
+//              loads its Q tiles by TMA once the previous unit's S MMAs have
+//              completed.
 // Tensor memory (512 columns, allocated once): per tile t at 256 t, O [0,128)
 // fp32 and two S buffers [128,192), [192,256) fp32, each overwritten in place
 // by its P as packed bf16 pairs. Issue order per tile S_0, S_1, PV_0, S_2,
@@ -45,10 +47,9 @@
 // than 2^8 (log2 domain), so O in tensor memory is rescaled rarely; O and the
 // row sum l always share the same reference max, so the final O / l is exact
 // up to rounding.
-// Shared memory: Q 2 x 32 KB (reloaded per unit once both issuers' last S
-// MMAs have completed), 3 x 32 KB K/V stages (K and V halves 8 KB each,
-// 128-byte swizzle, the canonical K-major / MN-major UMMA layouts), 2 x 32 KB
-// output staging (the Q tile layout).
+// Shared memory: Q 2 x 32 KB (reloaded per unit), 4 x 32 KB K/V stages (K and
+// V halves 8 KB each, 128-byte swizzle, the canonical K-major / MN-major UMMA
+// layouts), 2 x 16 KB output staging (half a tile each, the Q tile layout).
 // Every wait gives up after 2 s (PA_DEVERR_TIMEOUT) and its role stops; the
 // other roles' waits then run out in turn, and the CTA still frees its tensor
 // memory before it exits. Phase tracking: every mbarrier is waited on at most
