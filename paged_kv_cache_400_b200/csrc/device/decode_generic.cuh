@@ -16,8 +16,12 @@
 
 namespace pagedkv {
 
+// Up to 8 query heads per KV head the per-head state fits in 128 registers, so
+// the kernel is compiled for 4 resident CTAs per SM (which also lets the
+// compiler keep the smallest instances out of local memory); 16 heads need
+// more registers per thread.
 template <typename T, int D, int GMAX>
-__global__ void __launch_bounds__(128) decode_generic_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(128, GMAX <= 8 ? 4 : 1) decode_generic_kernel(DecodeParams p) {
   constexpr int NW = 4;
   constexpr int PER = D / 32;
   const int32_t part = blockIdx.x;
