@@ -127,14 +127,15 @@ __device__ __forceinline__ uint32_t tc_region(int kv, int half) { return (uint32
 
 // The launch enumerates work units, not a dense (unit, head, sequence) box:
 // sequence b brings ceil(n_b / U) units of U new tokens for each KV head, so
-// no CTA exists for the missing units of short sequences. Index idx runs over
-// the sequences in order, all KV heads of a sequence together, each head's
-// units last-first (the longest first). The calling warp finds idx's unit by a
-// prefix sum of the unit counts, 32 sequences per pass, loading one pass
-// ahead; sequences whose query range is malformed count no units (and set
-// PA_DEVERR_SEQLEN, from the lookup of idx 0, which scans every sequence).
-// Returns false when idx lies past the last unit (the grid size is an upper
-// bound).
+// no CTA exists for the missing units of short sequences. A sequence's units
+// are contiguous in the order, all its KV heads together, each head's units
+// last-first (the longest first). Up to kTcSortedSeqs sequences the sequences
+// go longest first (UnitOrder, below); past that in index order, looked up
+// here: the calling warp finds idx's unit by a prefix sum of the unit counts,
+// 32 sequences per pass, loading one pass ahead; sequences whose query range
+// is malformed count no units (and set PA_DEVERR_SEQLEN, from the lookup of
+// idx 0, which scans every sequence). Returns false when idx lies past the
+// last unit (the grid size is an upper bound).
 __device__ __forceinline__ bool find_unit(const PrefillParams& p, int32_t num_seqs, int32_t U, int32_t idx,
                                           TcUnit& u) {
   const int32_t lane = threadIdx.x & 31;
