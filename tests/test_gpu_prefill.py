@@ -118,6 +118,18 @@ def test_more_sequences_than_the_sorted_order():
     check_full(case)
 
 
+@pytest.mark.parametrize("nseq", [128, 129])
+def test_sorted_order_boundary(nseq):
+    # exactly the sorted order's 128 sequences (all four 32-sequence slots
+    # full) and one more (index order); many equal lengths, some empty
+    rng = np.random.default_rng(17 + nseq)
+    n = rng.integers(0, 48, size=nseq)
+    n[::7] = 16
+    ctx = np.where(np.arange(nseq) % 5 == 0, 0, rng.integers(0, 30, size=nseq))
+    case = wl.prefill_custom(f"order{nseq}", 17, ctx.tolist(), n.tolist(), 16, 8)
+    check_full(case)
+
+
 @pytest.mark.parametrize("where", [1, 40, 140])
 def test_malformed_query_ranges_flagged(where):
     # a decreasing query_start (n < 0) or a range past the last q row makes
