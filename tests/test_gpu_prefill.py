@@ -278,6 +278,57 @@ def test_repeated_calls_are_deterministic():
         assert torch.equal(out.view(torch.int16), again.view(torch.int16))
 
 
+def _prefill_args(case):
+    prep = prepare_prefill_step(case)
+    pool = case.make_pool(DEV)
+    k, v = case.make_kv_new(DEV)
+    pk.pa_reshape_and_cache(k, v, pool, torch.from_numpy(prep.slot_mapping).to(DEV))
+    return (case.make_q(DEV), pool, torch.from_numpy(prep.block_tables).to(DEV),
+            torch.from_numpy(prep.seq_lens).to(DEV), torch.from_numpy(prep.query_start).to(DEV),
+            case.scale, case.max_query_len)
+
+
+def test_concurrent_launches_on_two_streams():
+    # two launches in flight at once on two streams: each grid's running CTAs
+    # take only that grid's units, so both outputs equal their lone runs bit
+    # for bit
+    a = _prefill_args(wl.chunked_prefill_case(3, batch=12, chunk=256))
+    b = _prefill_args(wl.prefill_case(4, batch=24))
+    ref_a, ref_b = torch.zeros_like(a[0]), torch.zeros_like(b[0])
+    pk.pa_prefill(ref_a, *a)
+    pk.pa_prefill(ref_b, *b)
+    torch.cuda.synchronize()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    for _ in range(3):
+        got_a, got_b = torch.zeros_like(a[0]), torch.zeros_like(b[0])
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s1):
+            pk.pa_prefill(got_a, *a)
+        with torch.cuda.stream(s2):
+            pk.pa_prefill(got_b, *b)
+        torch.cuda.synchronize()
+        assert pk.pa_get_device_error() == 0
+        assert torch.equal(got_a.view(torch.int16), ref_a.view(torch.int16))
+        assert torch.equal(got_b.view(torch.int16), ref_b.view(torch.int16))
+
+
+def test_graph_replay_matches_eager():
+    args = _prefill_args(wl.prefill_custom("graph", 18, [0, 100, 7, 0], [300, 45, 1, 129], 32, 8))
+    ref = torch.zeros_like(args[0])
+    pk.pa_prefill(ref, *args)
+    torch.cuda.synchronize()
+    out = torch.zeros_like(args[0])
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        pk.pa_prefill(out, *args)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert pk.pa_get_device_error() == 0
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+
+
 def test_last_row_matches_decode():
     # the newest token's prefill row attends to the whole sequence, as decode does
     case = wl.prefill_custom("vs_decode", 6, [100, 0, 31], [50, 77, 1], 32, 8)
