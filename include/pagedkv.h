@@ -253,9 +253,14 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* kv_pool,
  * taken later are skipped. Allocates nothing.
  * Kernel: tcgen05 MMAs with tensor-memory accumulators, two 128-row query
  * tiles per work unit, about one persistent CTA per SM taking units in launch
- * order. There is no run-time kernel choice: the mma.sync kernel exists only
- * in a separate comparison build of this library (compiled with
- * PA_PREFILL_MMA_SYNC; same results within rounding).
+ * order (longest sequences first, up to 128 sequences) by cancelling CTAs of
+ * the same launch that have not started. Launches on different streams may
+ * run at the same time: each takes only its own units. The call may be
+ * captured in a CUDA graph; make one call on the device before the first
+ * capture (it sets the kernel's shared-memory limit once per device). There is
+ * no run-time kernel choice: the mma.sync kernel exists only in a separate
+ * comparison build of this library (compiled with PA_PREFILL_MMA_SYNC; same
+ * results within rounding).
  */
 pa_status pa_prefill(void* out, const void* q, const void* kv_pool,
                      const int32_t* block_tables, int32_t max_blocks_per_seq,
