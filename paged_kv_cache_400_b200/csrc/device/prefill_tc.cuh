@@ -136,18 +136,28 @@ __device__ __forceinline__ uint32_t tc_region(int kv, int half) { return (uint32
 // is malformed count no units (and set PA_DEVERR_SEQLEN, from the lookup of
 // idx 0, which scans every sequence). Returns false when idx lies past the
 // last unit (the grid size is an upper bound).
+// A CTA's successive lookups come in increasing idx order (cancelled CTAs are
+// handed out in launch order), so the scan resumes at the pass that held the
+// previous unit (cursor: that pass's first sequence and the units before it):
+// a CTA scans the sequences about once per launch, not once per unit.
+struct UnitCursor {
+  int32_t s0 = 0;    // first sequence of the pass to start at
+  int32_t base = 0;  // units of the sequences before it, times the KV heads
+};
+
 __device__ __forceinline__ bool find_unit(const PrefillParams& p, int32_t num_seqs, int32_t U, int32_t idx,
-                                          TcUnit& u) {
+                                          TcUnit& u, UnitCursor& cur) {
   const int32_t lane = threadIdx.x & 31;
-  int32_t base = 0;  // units of the sequences before this pass, times the KV heads
+  if (idx == 0 || idx < cur.base) cur = UnitCursor{};  // idx 0 scans every sequence (error check)
+  int32_t base = cur.base;
   bool any_bad = false, found = false;
   int32_t a_nx = 0, e_nx = 0, l_nx = 0;
-  if (lane < num_seqs) {
-    a_nx = __ldg(p.query_start + lane);
-    e_nx = __ldg(p.query_start + lane + 1);
-    l_nx = __ldg(p.seq_lens + lane);
+  if (cur.s0 + lane < num_seqs) {
+    a_nx = __ldg(p.query_start + cur.s0 + lane);
+    e_nx = __ldg(p.query_start + cur.s0 + lane + 1);
+    l_nx = __ldg(p.seq_lens + cur.s0 + lane);
   }
-  for (int32_t s0 = 0; s0 < num_seqs; s0 += 32) {
+  for (int32_t s0 = cur.s0; s0 < num_seqs; s0 += 32) {
     const int32_t s = s0 + lane;
     const int32_t a = a_nx, n = e_nx - a_nx, L = l_nx;
     if (s + 32 < num_seqs) {
@@ -178,6 +188,7 @@ __device__ __forceinline__ bool find_unit(const PrefillParams& p, int32_t num_se
       u.q0 = __shfl_sync(0xffffffffu, a, src);
       u.n = __shfl_sync(0xffffffffu, n, src);
       u.L = __shfl_sync(0xffffffffu, L, src);
+      if (!found) cur = UnitCursor{s0, base};
       found = true;
       if (idx != 0) return true;
     }
@@ -490,10 +501,11 @@ __global__ void __launch_bounds__(TcConfig<kQTiles>::kThreads, 1)
     // is malformed, or a wait has timed out somewhere in the grid (then the
     // remaining units are skipped; the error stays set until the host reads it).
     UnitOrder order;
+    UnitCursor cursor;
     const bool sorted = num_seqs <= kTcSortedSeqs;
     if (sorted) build_unit_order(p, num_seqs, U, order);
     auto resolve = [&](int32_t i, TcUnit& u) -> bool {
-      if (!(sorted ? find_unit_sorted(p, order, i, u) : find_unit(p, num_seqs, U, i, u))) return false;
+      if (!(sorted ? find_unit_sorted(p, order, i, u) : find_unit(p, num_seqs, U, i, u, cursor))) return false;
       if (u.L < u.n || (int64_t)u.L > (int64_t)p.max_blocks * 16) {
         if (u.unit == 0 && u.g == 0 && lane == 0) raise_device_error(PA_DEVERR_SEQLEN);
         return false;

@@ -118,6 +118,16 @@ def test_more_sequences_than_the_sorted_order():
     check_full(case)
 
 
+def test_a_thousand_short_sequences():
+    # 1000 sequences past the sorted order: every CTA's lookups resume from
+    # the pass of its previous unit (31 passes of 32 sequences)
+    rng = np.random.default_rng(19)
+    n = rng.integers(0, 40, size=1000)
+    ctx = rng.integers(0, 24, size=1000)
+    case = wl.prefill_custom("thousand", 19, ctx.tolist(), n.tolist(), 16, 8)
+    check_full(case)
+
+
 @pytest.mark.parametrize("nseq", [128, 129])
 def test_sorted_order_boundary(nseq):
     # exactly the sorted order's 128 sequences (all four 32-sequence slots
