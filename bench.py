@@ -72,7 +72,7 @@ def parse_args():
     ap.add_argument("--prefill-cpu-seconds", type=float, default=4.0,
                     help="bounded oracle sample of the chunked-prefill leg")
     ap.add_argument("--no-prefill-leg", action="store_true",
-                    help="gqa: skip the chunked-prefill measurement added to the line")
+                    help="gqa: skip the prefill measurements added to the line (chunked, whole prompts)")
     ap.add_argument("--kv-util-jsonl", default=None,
                     help="trace: write each step's KV-cache utilisation record to this file")
     return ap.parse_args()
@@ -489,10 +489,13 @@ def run_ours(args, rank, world, dist):
     e2e_s = max_over_ranks((p1 - p0) / E, dist, dev)
     assert pk.pa_get_device_error() == 0
 
-    # the chunked-prefill leg (the step on the other side of decode), every rank
-    prefill_line = None
+    # the prefill legs (the step on the other side of decode): chunked prefill
+    # and whole prompts, every rank
+    prefill_line = prompts_line = None
     if args.workload == "gqa" and not args.no_prefill_leg:
         prefill_line = measure_prefill(args, rank, world, dist, True, max(K, 10), args.warmup,
+                                       None if args.no_cpu_baseline else args.prefill_cpu_seconds)
+        prompts_line = measure_prefill(args, rank, world, dist, False, max(K, 10), args.warmup,
                                        None if args.no_cpu_baseline else args.prefill_cpu_seconds)
 
     if rank != 0:
@@ -551,6 +554,8 @@ def run_ours(args, rank, world, dist):
         line["unique_kv_gbs"] = ub / (ms_per_step / 1e3) / 1e9
     if prefill_line is not None:
         line["chunked_prefill"] = prefill_line
+    if prompts_line is not None:
+        line["prompts_prefill"] = prompts_line
     if not args.no_cpu_baseline and world == 1:
         done, el = oracle_sample(case, args.cpu_seconds)
         line["cpu_baseline"] = {
