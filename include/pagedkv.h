@@ -63,8 +63,9 @@ typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
 #define PA_DEVERR_BLOCK   2u  /* decode/copy: block id outside [0, num_blocks) */
 #define PA_DEVERR_SEQLEN  4u  /* decode: seq_len < 0, > max_seq_len, or beyond
                                  max_blocks_per_seq * 16                     */
-#define PA_DEVERR_TIMEOUT 8u  /* decode: a wait for staged data gave up after
-                                 2 s (the kernel returned instead of hanging) */
+#define PA_DEVERR_TIMEOUT 8u  /* decode/prefill: a wait for staged data gave
+                                 up after 2 s (the kernel returned instead of
+                                 hanging)                                    */
 
 /*
  * The KV pool of one attention layer: one contiguous device buffer
@@ -302,6 +303,16 @@ pa_status pa_copy_blocks_between(void* dst_pool, int32_t dst_num_blocks, const v
  * word was non-zero, PA_OK when zero.
  */
 pa_status pa_get_device_error(uint32_t* flags, void* stream);
+
+/*
+ * Self-test of the timeout path every kernel's waits share: one thread waits
+ * on an mbarrier that nothing arrives at, with the same bounded wait as the
+ * kernels but a limit of limit_ns nanoseconds (1 .. 10^9), then sets
+ * PA_DEVERR_TIMEOUT and returns, leaving the context usable. Enqueued on
+ * `stream`; read the bit with pa_get_device_error. A limit outside the range
+ * returns PA_ERR_INVALID_ARG.
+ */
+pa_status pa_selftest_timeout(uint64_t limit_ns, void* stream);
 
 /* Static text for a status code. */
 const char* pa_status_string(pa_status s);

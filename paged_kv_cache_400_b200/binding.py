@@ -79,6 +79,7 @@ def _declare(lib):
         "pa_append_decode": (i32, [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, f32, pa_pool_desc, vp, sz,
                                    i32, vp]),
         "pa_get_device_error": (i32, [C.POINTER(C.c_uint32), vp]),
+        "pa_selftest_timeout": (i32, [C.c_uint64, vp]),
         "pa_status_string": (C.c_char_p, [i32]),
         "pa_last_error": (C.c_char_p, []),
         "pa_bm_create": (i32, [i32, i32, _P32, C.POINTER(vp)]),
@@ -337,6 +338,12 @@ def pa_copy_blocks_between(dst_pool, src_pool, src, dst, stream=None):
     _check("pa_copy_blocks_between", lib().pa_copy_blocks_between(
         C.c_void_p(dst_pool.data_ptr()), dst_pool.shape[0], C.c_void_p(src_pool.data_ptr()), src_pool.shape[0],
         C.c_void_p(src.data_ptr()), C.c_void_p(dst.data_ptr()), n, desc, _stream(stream)))
+
+
+def pa_selftest_timeout(limit_ns: int, stream=None):
+    """One thread waits on a barrier nothing arrives at until its bounded
+    wait gives up after limit_ns, then sets PA_DEVERR_TIMEOUT."""
+    _check("pa_selftest_timeout", lib().pa_selftest_timeout(C.c_uint64(int(limit_ns)), _stream(stream)))
 
 
 def pa_get_device_error(stream=None) -> int:

@@ -433,6 +433,28 @@ pa_status pa_copy_blocks_between(void* dst_pool, int32_t dst_num_blocks, const v
   return launch_status("pa_copy_blocks_between");
 }
 
+namespace pagedkv {
+// One thread waits on a barrier nothing arrives at; the bounded wait gives up
+// after limit_ns and the error bit is raised as the kernels raise it.
+__global__ void selftest_timeout_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  if (!mbar_wait_bounded(&bar, 0, limit_ns)) raise_device_error(PA_DEVERR_TIMEOUT);
+}
+}  // namespace pagedkv
+
+pa_status pa_selftest_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1 || limit_ns > 1000000000ull)
+    return fail(PA_ERR_INVALID_ARG, "pa_selftest_timeout: limit %llu ns outside 1 .. 1e9",
+                (unsigned long long)limit_ns);
+  pagedkv::selftest_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(limit_ns);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_selftest_timeout: %s", cudaGetErrorString(e));
+  return PA_OK;
+}
+
 pa_status pa_get_device_error(uint32_t* flags, void* stream) {
   if (!flags) return fail(PA_ERR_INVALID_ARG, "pa_get_device_error: flags is NULL");
   void* addr = nullptr;
