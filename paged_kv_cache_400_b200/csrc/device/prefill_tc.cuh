@@ -16,8 +16,9 @@
 // next units itself by cancelling CTAs that have not started (cluster launch
 // control), so about one CTA per SM runs, set up once, and one unit's start
 // (Q and first K/V loads, first S) and end (last PV, output stores) overlap
-// its neighbours' work instead of leaving the SM idle between CTAs. Units go
-// out longest sequence first, so the grid ends on short ones.
+// its neighbours' work instead of leaving the SM idle between CTAs. Up to 128
+// sequences the units go out longest sequence first, so the grid ends on short
+// ones; past that in sequence order.
 //
 // 416 threads in five roles:
 //   warps 0-3, 4-7  softmax, one warp group per query tile: thread r owns row
