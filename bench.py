@@ -504,7 +504,12 @@ def run_ours(args, rank, world, dist):
     step_avg = sum(step_ms) / K
     fused_bytes = nbytes["decode"] + nbytes["append"]
     achieved = fused_bytes / (step_avg / 1e3) / 1e9
-    traffic, traffic_src = recorded_traffic()
+    # the ncu record is of the batch-256 GQA launch (seed 0); other decode
+    # workloads carry none
+    if args.workload == "gqa" and args.batch == 256 and args.seed + rank == 0:
+        traffic, traffic_src = recorded_traffic()
+    else:
+        traffic, traffic_src = None, "captured for the batch-256 GQA workload only"
     kv_gbs = nbytes["kv"] / (ms_per_step / 1e3) / 1e9
     cfg = workload_description(case, prep.seq_lens)
     cfg["global_batch"] = B * world
@@ -971,8 +976,8 @@ def measure_prefill(args, rank, world, dist, chunked, K, warmup, cpu_seconds):
     kv_bytes = int(sum(int(c) + int(n) for c, n in zip(case.ctx_lens, case.query_lens))) * 2 * \
         case.num_kv_heads * case.head_dim * 2
     traffic, traffic_src = None, ("mma.sync kernel: not captured" if mma_sync else
-                                  "captured at 64 sequences only")
-    if args.prefill_kernel == "tcgen05" and pb == 64:
+                                  "captured at 64 sequences (seed 0) only")
+    if args.prefill_kernel == "tcgen05" and pb == 64 and args.seed + rank == 0:
         traffic, traffic_src = recorded_traffic(
             os.path.join(ROOT, "profiles", f"prefill_tc_{'chunked' if chunked else 'prompts'}_b64.json"),
             PREFILL_KERNEL_SOURCES)
