@@ -60,6 +60,9 @@ constexpr int kStagedWarps = 4;
 constexpr int kStagedStages = 2;                 // per warp
 constexpr int kStageBytes = 8192;                // K + V of one block, one KV head
 constexpr int kStagedSmem = kStagedWarps * kStagedStages * kStageBytes + 1024;
+constexpr int kMergeRow = 128 + 8;  // floats per row of the warps' merge buffer
+static_assert(kStagedWarps * 16 * kMergeRow * 4 <= kStagedWarps * kStagedStages * kStageBytes,
+              "the merge buffer reuses the consumed stages");
 constexpr uint64_t kWaitLimitNs = 2000000000ull; // 2 s
 
 // Byte offset in a stage of the 16-byte chunk `chunk16` (0..15, head dims
@@ -380,7 +383,10 @@ __device__ __forceinline__ void decode_partition(const CUtensorMap& tmap, const 
 
   // ---- merge the four warps' states ------------------------------------------
   __syncthreads();  // every warp has consumed all its stages
-  float* so = reinterpret_cast<float*>(smem);  // [4 warps][16 rows][128] fp32
+  // [4 warps][16 rows][128] fp32, rows kMergeRow floats apart: the 8 extra
+  // words shift each row by 8 banks, so a warp's 8-row stores (and the
+  // merge's reads) spread over all banks
+  float* so = reinterpret_cast<float*>(smem);
   if constexpr (kMMA) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
@@ -394,8 +400,8 @@ __device__ __forceinline__ void decode_partition(const CUtensorMap& tmap, const 
     }
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
-      float* r0 = so + (warp * 16 + gid) * 128 + 8 * n + 2 * tig;
-      float* r1 = so + (warp * 16 + gid + 8) * 128 + 8 * n + 2 * tig;
+      float* r0 = so + (warp * 16 + gid) * kMergeRow + 8 * n + 2 * tig;
+      float* r1 = so + (warp * 16 + gid + 8) * kMergeRow + 8 * n + 2 * tig;
       *reinterpret_cast<float2*>(r0) = make_float2(o[n][0], o[n][1]);
       *reinterpret_cast<float2*>(r1) = make_float2(o[n][2], o[n][3]);
     }
@@ -408,7 +414,7 @@ __device__ __forceinline__ void decode_partition(const CUtensorMap& tmap, const 
       red_l[warp][0] = l0;
     }
     if (lane < 16) {
-      float* r = so + warp * 16 * 128 + 8 * lane;
+      float* r = so + warp * 16 * kMergeRow + 8 * lane;
       *reinterpret_cast<float4*>(r) = make_float4(acc[0], acc[1], acc[2], acc[3]);
       *reinterpret_cast<float4*>(r + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
@@ -426,7 +432,7 @@ __device__ __forceinline__ void decode_partition(const CUtensorMap& tmap, const 
     for (int w = 0; w < kStagedWarps; ++w) {
       const float e = exp2f(red_m[w][h] - M);  // 0 for a warp that had no block
       Ls = fmaf(red_l[w][h], e, Ls);
-      A = fmaf(so[(w * 16 + h) * 128 + d], e, A);
+      A = fmaf(so[(w * 16 + h) * kMergeRow + d], e, A);
     }
     const size_t bh = (size_t)b * H + (size_t)g * G + h;
     if (nparts == 1) {
