@@ -4,7 +4,7 @@
 // "大模型推理性能优化：PagedAttention与Continuous Batching原理与实践" §2.2 names the
 // scatter of new K/V into scattered pages as one of the two memory operations
 // PagedAttention kernels must do well; "vLLM 原理" / 工作原理 §2 gives the
-// position -> (page, row) mapping. Both kernels are plain 16-byte copies: every
+// position -> (page, row) mapping. The kernels are plain 16-byte copies: every
 // thread moves one 16-byte chunk, consecutive threads take consecutive chunks
 // of one (token, K|V, head) row, so each row is one coalesced run on both sides.
 #pragma once
@@ -13,33 +13,31 @@
 
 namespace pagedkv {
 
-// One thread per 16-byte chunk; item i = ((t * 2 + kv) * Hkv + h) * C + c,
-// C = chunks per (token, head) row.
+// One thread per 16-byte chunk. CTA (x, h, kv) covers 256 consecutive chunks
+// of the rows (token t, K|V kv, KV head h) in token order, kChunks chunks per
+// row (a compile-time count, so the index arithmetic is a shift and a mask;
+// the head and K|V come from the grid, not from a division).
+template <int kChunks>
 __global__ void __launch_bounds__(256)
 append_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, uint4* __restrict__ pool,
-              const int64_t* __restrict__ slots, int32_t num_tokens, int32_t num_kv_heads,
-              int32_t chunks_per_row, int64_t num_slots) {
-  const int64_t total = (int64_t)num_tokens * 2 * num_kv_heads * chunks_per_row;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
-    const int32_t c = (int32_t)(i % chunks_per_row);
-    int64_t r = i / chunks_per_row;
-    const int32_t h = (int32_t)(r % num_kv_heads);
-    r /= num_kv_heads;
-    const int32_t kv = (int32_t)(r & 1);
-    const int64_t t = r >> 1;
-    const int64_t s = __ldg(slots + t);
-    if (s < 0) continue;  // padding
-    if (s >= num_slots) {
-      if (c == 0 && h == 0 && kv == 0) raise_device_error(PA_DEVERR_SLOT);
-      continue;
-    }
-    const int64_t blk = s >> 4;
-    const int32_t row = (int32_t)(s & 15);
-    const uint4* src = (kv ? v : k) + (t * num_kv_heads + h) * chunks_per_row + c;
-    uint4* dst = pool + (((blk * 2 + kv) * num_kv_heads + h) * 16 + row) * chunks_per_row + c;
-    *dst = __ldg(src);
+              const int64_t* __restrict__ slots, int32_t num_tokens, int32_t num_kv_heads, int64_t num_slots) {
+  const int32_t h = blockIdx.y;
+  const int32_t kv = blockIdx.z;
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t t = e / kChunks;
+  const int32_t c = (int32_t)(e % kChunks);
+  if (t >= num_tokens) return;
+  const int64_t s = __ldg(slots + t);
+  if (s < 0) return;  // padding
+  if (s >= num_slots) {
+    if (c == 0 && h == 0 && kv == 0) raise_device_error(PA_DEVERR_SLOT);
+    return;
   }
+  const int64_t blk = s >> 4;
+  const int32_t row = (int32_t)(s & 15);
+  const uint4* src = (kv ? v : k) + (t * num_kv_heads + h) * kChunks + c;
+  uint4* dst = pool + (((blk * 2 + kv) * num_kv_heads + h) * 16 + row) * kChunks + c;
+  *dst = __ldg(src);
 }
 
 // One CTA per pair; the CTA copies the whole block as 16-byte chunks.

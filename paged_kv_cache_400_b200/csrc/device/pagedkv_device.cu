@@ -171,14 +171,20 @@ pa_status pa_reshape_and_cache(const void* k, const void* v, void* kv_pool,
     return fail(PA_ERR_INVALID_ARG, "pa_reshape_and_cache: NULL pointer");
   if (!aligned16(k) || !aligned16(v) || !aligned16(kv_pool))
     return fail(PA_ERR_INVALID_ARG, "pa_reshape_and_cache: k, v and kv_pool must be 16-byte aligned");
-  const int32_t chunks = (int32_t)(pool.head_dim * elem_size(pool.dtype) / 16);
-  const int64_t total = (int64_t)num_tokens * 2 * pool.num_kv_heads * chunks;
-  const int64_t want = (total + 255) / 256;
-  const int32_t grid = (int32_t)(want < 65535 * 16 ? want : 65535 * 16);
-  pagedkv::append_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(
-      reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v),
-      reinterpret_cast<uint4*>(kv_pool), slot_mapping, num_tokens, pool.num_kv_heads, chunks,
-      (int64_t)pool.num_blocks * PA_BLOCK_SIZE);
+  const int32_t chunks = (int32_t)(pool.head_dim * elem_size(pool.dtype) / 16);  // 8, 16 or 32
+  const int64_t per_rows = (int64_t)num_tokens * chunks;  // chunks of one (K|V, head) across the tokens
+  const dim3 grid((unsigned)((per_rows + 255) / 256), (unsigned)pool.num_kv_heads, 2);
+  const uint4* k4 = reinterpret_cast<const uint4*>(k);
+  const uint4* v4 = reinterpret_cast<const uint4*>(v);
+  uint4* p4 = reinterpret_cast<uint4*>(kv_pool);
+  const int64_t num_slots = (int64_t)pool.num_blocks * PA_BLOCK_SIZE;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (chunks == 8)
+    pagedkv::append_kernel<8><<<grid, 256, 0, st>>>(k4, v4, p4, slot_mapping, num_tokens, pool.num_kv_heads, num_slots);
+  else if (chunks == 16)
+    pagedkv::append_kernel<16><<<grid, 256, 0, st>>>(k4, v4, p4, slot_mapping, num_tokens, pool.num_kv_heads, num_slots);
+  else
+    pagedkv::append_kernel<32><<<grid, 256, 0, st>>>(k4, v4, p4, slot_mapping, num_tokens, pool.num_kv_heads, num_slots);
   return launch_status("pa_reshape_and_cache");
 }
 
