@@ -520,8 +520,12 @@ __global__ void __launch_bounds__(128) decode_staged_kernel(const __grid_constan
 // sequence's last partition by decreasing size (counting sort on the size in
 // blocks). Also raises PA_DEVERR_SEQLEN for bad lengths, writes zeros for
 // sequences of length 0, and resets the item counter.
+// Launched as a programmatic dependent of the kernel before it in the stream
+// (often the previous step's decode), so its launch overlaps that kernel;
+// nothing is read or written before that kernel has completed.
 constexpr int kPlanThreads = 1024;
 constexpr int kMaxPartitionBlocks = 128;  // partitions of at most 2048 tokens
+static_assert(kMaxPartitionBlocks <= 4 * 32, "the plan's scan covers 4 sizes per lane of one warp");
 
 __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams p) {
   __shared__ int32_t cnt[kMaxPartitionBlocks + 1];
@@ -529,6 +533,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
   // the decode CTAs may start (and set up) now; they wait for this grid's
   // completion before reading the list
   grid_dependents_launch();
+  grid_dependency_wait();  // the kernel before this one is complete (inputs written, old list read)
   const int32_t SB = p.partition_tokens >> 4;  // blocks per full partition (<= kMaxPartitionBlocks)
   for (int32_t i = threadIdx.x; i <= SB; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
@@ -545,14 +550,35 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(DecodeParams 
     atomicAdd(&cnt[r], 1);
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int32_t acc = 0;
-    for (int32_t sz = SB; sz >= 1; --sz) {
-      off[sz] = acc;
-      acc += cnt[sz];
+  if (threadIdx.x < 32) {
+    // exclusive prefix sum of the counts in decreasing size (positions
+    // 0 .. SB-1 hold sizes SB .. 1): lane l sums positions 4l .. 4l+3, a
+    // warp scan adds the lanes before it
+    const int32_t lane = threadIdx.x;
+    int32_t c[4], own = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int32_t sz = SB - (4 * lane + k);
+      c[k] = sz >= 1 ? cnt[sz] : 0;
+      own += c[k];
     }
-    p.work_header[0] = acc;
-    p.work_header[1] = 0;
+    int32_t incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int32_t run = incl - own;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int32_t sz = SB - (4 * lane + k);
+      if (sz >= 1) off[sz] = run;
+      run += c[k];
+    }
+    if (lane == 31) {
+      p.work_header[0] = incl;
+      p.work_header[1] = 0;
+    }
   }
   __syncthreads();
   for (int32_t b = threadIdx.x; b < p.num_seqs; b += blockDim.x) {
@@ -644,8 +670,16 @@ inline pa_status launch_staged_bf16_d128(const DecodeParams& p, cudaStream_t st)
   pa_status s = encode_pool_map(p.pool, p.num_kv_heads, p.num_blocks, &map);
   if (s != PA_OK) return s;
   if (p.work_items != nullptr) {
-    decode_plan_kernel<<<1, kPlanThreads, 0, st>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(kPlanThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_plan_kernel, p);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode (plan): launch failed: %s", cudaGetErrorString(e));
   }
   const bool append = p.k_new != nullptr;
@@ -654,9 +688,8 @@ inline pa_status launch_staged_bf16_d128(const DecodeParams& p, cudaStream_t st)
   else if (!append) s = launch_staged_variant<true, false>(map, p, st);
   else s = launch_staged_variant<true, true>(map, p, st);
   if (s != PA_OK) return s;
-  cudaError_t e = cudaSuccess;
   if (p.max_partitions <= 1) return PA_OK;
-  e = launch_partition_merge<__nv_bfloat16, 128>(p, st);
+  cudaError_t e = launch_partition_merge<__nv_bfloat16, 128>(p, st);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "pa_decode (merge): launch failed: %s", cudaGetErrorString(e));
   return PA_OK;
 }

@@ -190,6 +190,69 @@ def test_long_max_context_uses_the_work_list(max_seq_len):
     check_case(mha)
 
 
+def _work_list_case():
+    # 24 sequences up to 8192 tokens on 8 KV heads: four 2048-token partitions
+    # at most, the persistent decode over the plan kernel's work list
+    lens = [8192, 8191, 6145, 6144, 4097, 4096, 2049, 2048, 2047, 1, 16, 17, 3000, 5000, 7000, 100,
+            1500, 2500, 3500, 4500, 5500, 6500, 7500, 33]
+    return wl.custom_case("wl_graph", 19, lens, 8192, 32, 8, 128, "bf16", 512, 8192)
+
+
+def test_work_list_ignores_stale_workspace_contents():
+    # the plan kernel rewrites the item list, its count and the item counter
+    # on every call, so whatever the workspace holds on entry (here all bits
+    # set, then what a previous call left) gives the same output
+    case = _work_list_case()
+    prep, pool, ref, _ = check_case(case)
+    q = case.make_q(DEV)
+    bt = torch.from_numpy(prep.block_tables).to(DEV)
+    sl = torch.from_numpy(prep.seq_lens).to(DEV)
+    assert pk.pa_decode_partition_tokens(len(case.batch), 32, pool, 8192) == 2048
+    ws = pk.alloc_workspace(len(case.batch), case.num_heads, pool, case.max_seq_len)
+    ws.fill_(255)
+    for _ in range(2):
+        out = torch.empty_like(ref)
+        pk.pa_decode(out, q, pool, bt, sl, case.scale, case.max_seq_len, ws)
+        assert pk.pa_get_device_error() == 0
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+
+
+def test_work_list_decode_in_a_cuda_graph():
+    # the plan kernel is a programmatic dependent of the kernel before it:
+    # captured after a device copy (a non-kernel node before the plan) and
+    # twice in a row (the second plan follows the first call's merge kernel);
+    # replays are bit-identical to eager calls
+    case = _work_list_case()
+    prep, pool, ref, _ = check_case(case)
+    q_src = case.make_q(DEV)
+    q = torch.empty_like(q_src)
+    bt = torch.from_numpy(prep.block_tables).to(DEV)
+    sl = torch.from_numpy(prep.seq_lens).to(DEV)
+    ws = pk.alloc_workspace(len(case.batch), case.num_heads, pool, case.max_seq_len)
+    out1, out2 = torch.empty_like(ref), torch.empty_like(ref)
+    q.copy_(q_src)
+    pk.pa_decode(out1, q, pool, bt, sl, case.scale, case.max_seq_len, ws)   # eager first (attributes)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            q.copy_(q_src)
+            pk.pa_decode(out1, q, pool, bt, sl, case.scale, case.max_seq_len, ws)
+            pk.pa_decode(out2, q, pool, bt, sl, case.scale, case.max_seq_len, ws)
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(3):
+        out1.zero_()
+        out2.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert pk.pa_get_device_error() == 0
+        assert torch.equal(out1.view(torch.int16), ref.view(torch.int16))
+        assert torch.equal(out2.view(torch.int16), ref.view(torch.int16))
+    del g
+
+
 def test_single_token_sequences():
     case = wl.custom_case("ones", 12, [1] * 40, 128, 32, 8, 128, "bf16", 4, 64)
     _, _, out, _ = check_case(case)
