@@ -137,6 +137,24 @@ def test_workspace_size_is_deterministic_and_zero_for_one_partition():
     assert bd.lib().pa_decode_workspace_size(0, 2, p, 100) == 0
 
 
+@pytest.mark.parametrize("B,H,Hkv,D,max_len", [
+    (256, 32, 8, 128, 8192), (64, 32, 32, 128, 8192), (3, 32, 8, 128, 65536), (7, 12, 3, 64, 20000),
+    (1, 32, 8, 128, 131072), (1000, 16, 16, 128, 4096),
+])
+def test_workspace_covers_every_region_the_kernels_write(B, H, Hkv, D, max_len):
+    # the split-KV partial accumulators [B][H][P][D] fp32 and (m, l) pairs
+    # [B][H][P][2] fp32, and from 4 partitions on the work list [B][P] int32 and
+    # its counters: a workspace of the reported size must hold all of them
+    p = pool(num_blocks=4096, heads=Hkv, dim=D)
+    S = bd.lib().pa_decode_partition_tokens(B, H, p, max_len)
+    assert S % 16 == 0 and 128 <= S <= 2048
+    P = (max_len + S - 1) // S
+    need = B * H * P * D * 4 + B * H * P * 2 * 4 + (B * P * 4 + 2 * 4 if P >= 4 else 0)
+    size = bd.lib().pa_decode_workspace_size(B, H, p, max_len)
+    assert (size == 0) == (P <= 1)
+    assert size >= need
+
+
 def test_bm_errors_are_statuses():
     bm = bd.BlockManager(4)
     with pytest.raises(bd.PagedKVError) as e:
