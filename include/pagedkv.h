@@ -149,7 +149,8 @@ int32_t pa_decode_partition_tokens(int32_t num_seqs, int32_t num_heads,
  *       > max_blocks_per_seq*16 writes zeros and sets PA_DEVERR_SEQLEN.
  * A table entry outside [0, num_blocks) is not read; its tokens count as
  *       zero vectors and PA_DEVERR_BLOCK is set.
- * max_seq_len: host-known upper bound on seq_lens (sets the partition count).
+ * max_seq_len: host-known upper bound on seq_lens (sets the partition count;
+ *       a bound needing more than 65535 partitions is PA_ERR_UNSUPPORTED).
  * workspace: device, >= pa_decode_workspace_size(...) bytes, 256-byte aligned;
  *       contents on entry are ignored; must not be used by another call that
  *       overlaps this one on the GPU.

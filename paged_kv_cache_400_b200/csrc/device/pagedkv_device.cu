@@ -67,14 +67,17 @@ int32_t partition_tokens_for(int32_t num_seqs, const pa_pool_desc& pool, int32_t
   int32_t S = PA_PARTITION_TOKENS;
   const int64_t pairs = (int64_t)num_seqs * pool.num_kv_heads;
   const int64_t want = 4 * (int64_t)pagedkv::device_sm_count();
-  while (S > 128 && pairs * ((max_seq_len + S - 1) / S) < want) S /= 2;
+  while (S > 128 && pairs * (((int64_t)max_seq_len + S - 1) / S) < want) S /= 2;
   return S;
 }
 
+// The persistent decode's work items hold the partition index in 16 bits.
+constexpr int64_t kMaxPartitions = 65535;
+
 // Host-side checks shared by pa_decode, pa_append_decode and
 // pa_decode_noalloc, in this order: pool, sizes, head group, table width,
-// scale, then (for a non-empty batch) pointers and alignment. The workspace is
-// checked by the caller afterwards.
+// scale, then (for a non-empty batch) the partition count, pointers and
+// alignment. The workspace is checked by the caller afterwards.
 pa_status check_decode_args(const char* fn, const void* out, const void* q, const void* kv_pool,
                             const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* seq_lens,
                             int32_t num_seqs, int32_t num_heads, float scale, const pa_pool_desc& pool,
@@ -94,6 +97,10 @@ pa_status check_decode_args(const char* fn, const void* out, const void* q, cons
     return fail(PA_ERR_INVALID_ARG, "%s: max_seq_len %d > max_blocks_per_seq * 16", fn, max_seq_len);
   if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "%s: scale is not finite", fn);
   if (num_seqs == 0) return PA_OK;
+  const int32_t S = partition_tokens_for(num_seqs, pool, max_seq_len > 0 ? max_seq_len : 1);
+  if (((int64_t)max_seq_len + S - 1) / S > kMaxPartitions)
+    return fail(PA_ERR_UNSUPPORTED, "%s: max_seq_len %d needs more than %lld partitions of %d tokens", fn,
+                max_seq_len, (long long)kMaxPartitions, S);
   if (!out || !q || !kv_pool || !block_tables || !seq_lens) return fail(PA_ERR_INVALID_ARG, "%s: NULL pointer", fn);
   if (!aligned16(out) || !aligned16(q) || !aligned16(kv_pool))
     return fail(PA_ERR_INVALID_ARG, "%s: out, q and kv_pool must be 16-byte aligned", fn);
@@ -109,7 +116,7 @@ WorkspaceLayout workspace_layout(int32_t num_seqs, int32_t num_heads, const pa_p
                                  int32_t max_seq_len) {
   WorkspaceLayout w{0, 0, 0, 0, 0, 0};
   const int32_t S = partition_tokens_for(num_seqs, pool, max_seq_len);
-  w.partitions = (max_seq_len + S - 1) / S;
+  w.partitions = (int32_t)(((int64_t)max_seq_len + S - 1) / S);
   if (w.partitions <= 1) return w;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   const size_t units = (size_t)num_seqs * num_heads * w.partitions;

@@ -68,6 +68,25 @@ def test_decode_rejects_bad_arguments_on_host():
     assert L.pa_decode(None, None, None, None, 4, None, 0, 2, 0.1, p, None, 0, 16, None) == 0
 
 
+def test_decode_rejects_more_partitions_than_a_work_item_holds():
+    # the persistent decode keeps a partition index in 16 bits: a bound that
+    # needs more than 65535 partitions is refused on the host (status 2),
+    # before the workspace is looked at; 65535 itself passes that check
+    L = bd.lib()
+    vp = C.c_void_p(16)  # never dereferenced: rejected before use
+    p = pool(num_blocks=1 << 20, heads=8)
+    S = L.pa_decode_partition_tokens(1, 32, p, 140_000_000)
+    assert S == 2048
+    too_long = 65536 * S - 100
+    assert L.pa_decode(vp, vp, vp, vp, too_long // 16 + 1, vp, 1, 32, 0.1, p, None, 0, too_long, None) == 2
+    assert b"partitions" in L.pa_last_error()
+    assert L.pa_append_decode(vp, vp, vp, vp, vp, vp, vp, too_long // 16 + 1, vp, 1, 32, 0.1, p, None, 0,
+                              too_long, None) == 2
+    fits = 65535 * S
+    # the largest bound that fits: the next check (the missing workspace) answers
+    assert L.pa_decode(vp, vp, vp, vp, fits // 16, vp, 1, 32, 0.1, p, None, 0, fits, None) == 9
+
+
 def test_noalloc_reports_argument_errors_before_its_size_limit():
     """pa_decode_noalloc returns pa_decode's own argument errors even for a
     shape beyond its fixed array; only valid arguments reach the size check."""
